@@ -1,0 +1,209 @@
+"""The oracle: plain, slow, fp64 CPU exact attention.  TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline and reference
+legs may import this package.  The CUDA product path (``io_aware_exact_16_b200``) never
+imports it, and the two share no code: this package reads the same seeded bf16 inputs from
+``workloads`` and nothing else.
+
+Two independent implementations of the same definition live here:
+
+* ``oracle.c`` (built into ``liboracle.so``): the definition of attention written out row by
+  row in fp64 (FlashAttention (DE), "Problematik der Standard-Attention"), with the ordinary
+  derivative for the backward pass.  This is THE oracle.
+* ``twin.py``: the same definition as whole-matrix numpy float64 expressions, used by the
+  pin tests as a second, independently written implementation.
+
+Both take the exact fp64 values of the bf16 inputs.  Every function is pinned by
+``tests/test_oracle_pins.py`` against closed forms, invariances, finite differences and
+torch's own float64 attention (see the pins listed there).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_SO = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+_dp = ctypes.POINTER(ctypes.c_double)
+_ip = ctypes.POINTER(ctypes.c_int)
+
+
+def build(force: bool = False) -> str:
+    """Compile ``oracle.c`` into ``liboracle.so`` next to it (plain gcc, -O2, pthreads)."""
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-Wall", "-Wextra", "-fPIC", "-shared", "-o", _SO, _SRC,
+               "-lpthread", "-lm"]
+        subprocess.run(cmd, check=True)
+    return _SO
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        lib.oracle_attention_fwd.argtypes = [_dp, _dp, _dp, ctypes.c_int, ctypes.c_int,
+                                             ctypes.c_double, ctypes.c_int, ctypes.c_int, _dp, _dp]
+        lib.oracle_attention_fwd_rows.argtypes = [_dp, _dp, _dp, ctypes.c_int, ctypes.c_int,
+                                                  ctypes.c_double, ctypes.c_int, ctypes.c_int,
+                                                  _ip, ctypes.c_int, _dp, _dp]
+        lib.oracle_attention_probs.argtypes = [_dp, _dp, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_double, ctypes.c_int, ctypes.c_int, _dp]
+        lib.oracle_attention_bwd.argtypes = [_dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int,
+                                             ctypes.c_double, ctypes.c_int, ctypes.c_int,
+                                             _dp, _dp, _dp, _dp, _dp, _dp]
+        lib.oracle_attention_bwd_rows.argtypes = [_dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int,
+                                                  ctypes.c_double, ctypes.c_int, ctypes.c_int,
+                                                  _ip, ctypes.c_int, _ip, ctypes.c_int,
+                                                  _dp, _dp, _dp]
+        lib.oracle_set_threads.argtypes = [ctypes.c_int]
+        lib.oracle_get_threads.restype = ctypes.c_int
+        for name in ("oracle_attention_fwd", "oracle_attention_fwd_rows", "oracle_attention_probs",
+                     "oracle_attention_bwd", "oracle_attention_bwd_rows"):
+            getattr(lib, name).restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def set_threads(n: int) -> None:
+    """Number of CPU threads the oracle spreads rows over (0 = every online core)."""
+    _load().oracle_set_threads(int(n))
+
+
+def get_threads() -> int:
+    return int(_load().oracle_get_threads())
+
+
+def as_f64(x) -> np.ndarray:
+    """Exact fp64 copy of a bf16/fp32/fp64 torch tensor or numpy array (C-contiguous)."""
+    if hasattr(x, "detach"):
+        import torch  # only for the dtype conversion of torch inputs
+        x = x.detach().to("cpu", torch.float64).numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray):
+    assert a.dtype == np.float64 and a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(_dp)
+
+
+def _iptr(a: np.ndarray):
+    assert a.dtype == np.int32 and a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(_ip)
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != 0:
+        raise RuntimeError(f"oracle: {what} rejected its arguments")
+
+
+def head_fwd(q, k, v, scale: float, causal: bool, L: Optional[int] = None):
+    """One head: q, k, v ``[N, d]`` -> (O ``[N, d]``, lse ``[N]``) in fp64."""
+    q, k, v = as_f64(q), as_f64(k), as_f64(v)
+    N, d = q.shape
+    L = N if L is None else int(L)
+    O = np.empty((N, d), np.float64)
+    lse = np.empty((N,), np.float64)
+    _check(_load().oracle_attention_fwd(_ptr(q), _ptr(k), _ptr(v), N, d, float(scale),
+                                        int(bool(causal)), L, _ptr(O), _ptr(lse)), "fwd")
+    return O, lse
+
+
+def head_fwd_rows(q, k, v, rows: Sequence[int], scale: float, causal: bool,
+                  L: Optional[int] = None):
+    """One head, only the listed query rows: (O ``[len(rows), d]``, lse ``[len(rows)]``)."""
+    q, k, v = as_f64(q), as_f64(k), as_f64(v)
+    N, d = q.shape
+    L = N if L is None else int(L)
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+    O = np.empty((len(r), d), np.float64)
+    lse = np.empty((len(r),), np.float64)
+    _check(_load().oracle_attention_fwd_rows(_ptr(q), _ptr(k), _ptr(v), N, d, float(scale),
+                                             int(bool(causal)), L, _iptr(r), len(r), _ptr(O),
+                                             _ptr(lse)), "fwd_rows")
+    return O, lse
+
+
+def head_probs(q, k, scale: float, causal: bool, L: Optional[int] = None) -> np.ndarray:
+    """One head: the probability matrix P ``[N, N]`` (zero where a key is masked)."""
+    q, k = as_f64(q), as_f64(k)
+    N, d = q.shape
+    L = N if L is None else int(L)
+    P = np.empty((N, N), np.float64)
+    _check(_load().oracle_attention_probs(_ptr(q), _ptr(k), N, d, float(scale),
+                                          int(bool(causal)), L, _ptr(P)), "probs")
+    return P
+
+
+def head_bwd(q, k, v, do, scale: float, causal: bool, L: Optional[int] = None):
+    """One head: -> dict with dq, dk, dv, o, lse, D (all fp64)."""
+    q, k, v, do = as_f64(q), as_f64(k), as_f64(v), as_f64(do)
+    N, d = q.shape
+    L = N if L is None else int(L)
+    out = {name: np.empty((N, d), np.float64) for name in ("dq", "dk", "dv", "o")}
+    out["lse"] = np.empty((N,), np.float64)
+    out["D"] = np.empty((N,), np.float64)
+    _check(_load().oracle_attention_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(do), N, d, float(scale),
+                                        int(bool(causal)), L, _ptr(out["dq"]), _ptr(out["dk"]),
+                                        _ptr(out["dv"]), _ptr(out["o"]), _ptr(out["lse"]),
+                                        _ptr(out["D"])), "bwd")
+    return out
+
+
+def head_bwd_rows(q, k, v, do, qrows: Sequence[int], krows: Sequence[int], scale: float,
+                  causal: bool, L: Optional[int] = None):
+    """One head: dQ at the listed query rows, dK and dV at the listed key rows."""
+    q, k, v, do = as_f64(q), as_f64(k), as_f64(v), as_f64(do)
+    N, d = q.shape
+    L = N if L is None else int(L)
+    qr = np.ascontiguousarray(np.asarray(qrows, dtype=np.int32))
+    kr = np.ascontiguousarray(np.asarray(krows, dtype=np.int32))
+    dq = np.empty((max(len(qr), 1), d), np.float64)
+    dk = np.empty((max(len(kr), 1), d), np.float64)
+    dv = np.empty((max(len(kr), 1), d), np.float64)
+    _check(_load().oracle_attention_bwd_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(do), N, d,
+                                             float(scale), int(bool(causal)), L, _iptr(qr),
+                                             len(qr), _iptr(kr), len(kr), _ptr(dq), _ptr(dk),
+                                             _ptr(dv)), "bwd_rows")
+    return {"dq": dq[:len(qr)], "dk": dk[:len(kr)], "dv": dv[:len(kr)]}
+
+
+def _lengths(seqlens, B: int, N: int) -> list[int]:
+    if seqlens is None:
+        return [N] * B
+    return [int(x) for x in (seqlens.tolist() if hasattr(seqlens, "tolist") else seqlens)]
+
+
+def attention_fwd(q, k, v, scale: float, causal: bool, seqlens=None):
+    """Batched ``[B, H, N, d]`` inputs -> (O ``[B, H, N, d]``, lse ``[B, H, N]``), fp64."""
+    q, k, v = as_f64(q), as_f64(k), as_f64(v)
+    B, H, N, d = q.shape
+    Ls = _lengths(seqlens, B, N)
+    O = np.empty((B, H, N, d), np.float64)
+    lse = np.empty((B, H, N), np.float64)
+    for b in range(B):
+        for h in range(H):
+            O[b, h], lse[b, h] = head_fwd(q[b, h], k[b, h], v[b, h], scale, causal, Ls[b])
+    return O, lse
+
+
+def attention_bwd(q, k, v, do, scale: float, causal: bool, seqlens=None):
+    """Batched backward -> dict of ``[B, H, N, d]`` dq, dk, dv, o and ``[B, H, N]`` lse, D."""
+    q, k, v, do = as_f64(q), as_f64(k), as_f64(v), as_f64(do)
+    B, H, N, d = q.shape
+    Ls = _lengths(seqlens, B, N)
+    out = {n: np.empty((B, H, N, d), np.float64) for n in ("dq", "dk", "dv", "o")}
+    out["lse"] = np.empty((B, H, N), np.float64)
+    out["D"] = np.empty((B, H, N), np.float64)
+    for b in range(B):
+        for h in range(H):
+            r = head_bwd(q[b, h], k[b, h], v[b, h], do[b, h], scale, causal, Ls[b])
+            for n in out:
+                out[n][b, h] = r[n]
+    return out
