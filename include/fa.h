@@ -1,0 +1,132 @@
+/*
+ * fa.h -- C ABI of the exact-attention library for NVIDIA B200 (sm_100a).
+ *
+ * The library computes exact scaled-dot-product attention
+ *
+ *     O = softmax(scale * Q K^T [+ mask]) V
+ *
+ * (the formula of FlashAttention (DE), section "Problematik der Standard-Attention"), as one
+ * fused, tiled forward kernel that never writes the N x N score matrix to device memory
+ * (FlashAttention (DE), sections "Tiling und blockweise Verarbeitung", "Online-Softmax-
+ * Berechnung" and "Zusammenfassen von Operationen in einem CUDA-Kernel"), and a backward pass
+ * that keeps only the per-row log-sum-exp and recomputes the probabilities block by block
+ * (flash-attention glossary page, "Hoe werkt het?", item "Herberekening").
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout.     Q, K, V, O, dO, dQ, dK, dV are bf16, contiguous, shape [B, H, N, d]
+ *             (row-major: d fastest, then N, then H, then B).  lse is fp32 [B, H, N].
+ * Sizes.      B >= 1, H >= 1, 1 <= N, d in {64, 128}; B*H*N*d must fit in 2^31 elements.
+ * Mask.       causal != 0 hides key j from query i when j > i (top-left alignment, N queries
+ *             and N keys).  seqlens, when not NULL, is a DEVICE int32 array of B key lengths
+ *             L_b with 1 <= L_b <= N: keys j >= L_b of batch b are hidden from every query.
+ *             Both masks combine by AND.  Query rows i >= L_b are still computed (they attend
+ *             to the visible keys).  A length outside [1, N] is reported through the device
+ *             error flag as FA_ERR_INVALID_ARG and treated as clamped to [1, N].
+ * scale.      Multiplies Q K^T; must be finite and > 0 (1/sqrt(d) is the usual choice).
+ * Pointers.   Device pointers, 16-byte aligned, not aliasing one another (outputs never alias
+ *             inputs).  The caller allocates and owns every buffer, including the workspace.
+ * Streams.    `stream` is a cudaStream_t (NULL = the legacy default stream).  Every call only
+ *             validates its arguments and enqueues kernels on `stream`; FA_OK means
+ *             "validated and launched".  Errors found on the device (a bad length, a wait
+ *             that timed out) are recorded in a per-device error flag that
+ *             fa_check_device_error() reads.
+ * Errors.     No exception crosses the ABI.  A rejected call launches nothing and leaves every
+ *             output untouched.
+ * Device.     Requires a compute capability 10.0 GPU (B200); otherwise FA_ERR_UNSUPPORTED.
+ * Threads.    Calls may come from several host threads; calls on one stream run in order.
+ */
+#ifndef FA_H
+#define FA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+/* Same type as cudaStream_t, spelled without the CUDA headers. */
+typedef struct CUstream_st* fa_stream_t;
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1,  /* a NULL/misaligned pointer, a size or scale out of range      */
+    FA_ERR_UNSUPPORTED = 2,  /* head dim not 64/128, or the device is not sm_100             */
+    FA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed (launch, tensor map, ...)  */
+    FA_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up (reported by the flag)   */
+    FA_ERR_WORKSPACE = 5     /* fa_bwd: workspace NULL, misaligned or smaller than required */
+} fa_status;
+
+/*
+ * Forward pass.
+ *   q, k, v   in : bf16 [B, H, N, d]
+ *   o         out: bf16 [B, H, N, d]   O = softmax(scale * Q K^T + mask) V
+ *   lse       out: fp32 [B, H, N]      lse_i = ln sum_{j visible} exp(scale * q_i . k_j),
+ *                                      the "normalisation values" the backward pass keeps
+ *                                      (flash-attention glossary page, "Herberekening").
+ * One fused kernel: Q/K/V tiles staged through shared memory by TMA, Q K^T and P V on the
+ * tensor cores (tcgen05, accumulators in tensor memory), online softmax with a running row
+ * maximum and row sum (FlashAttention (DE), "Online-Softmax-Berechnung").  Allocates nothing.
+ */
+FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int H, int N, int d, float scale, int causal, const int* seqlens,
+                 fa_stream_t stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs for these sizes (0 if the sizes are invalid).
+ * The workspace holds D = rowsum(dO * O) (fp32 [B, H, N]), the fp32 dQ accumulator
+ * ([B, H, N_pad, d] with N_pad = N rounded up to 128), the per-(b, h, query-block) ordering
+ * counters of the deterministic dQ reduction and a tile counter.  Its contents need not be
+ * initialised; fa_bwd clears what it uses.
+ */
+FA_API size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Backward pass (training).  Recomputes P block by block from lse (flash-attention glossary
+ * page, "Herberekening") and forms the ordinary derivative of the forward formula:
+ *     dV = P^T dO,  dP = dO V^T,  D = rowsum(dO * O),  dS = P * (dP - D),
+ *     dK = scale * dS^T Q,  dQ = scale * dS K.
+ *   q, k, v, o, dO in : bf16 [B, H, N, d]; o is the forward output for the same inputs
+ *   lse            in : fp32 [B, H, N] from fa_fwd with the same inputs and mask
+ *   dq, dk, dv     out: bf16 [B, H, N, d], fully overwritten
+ *   workspace      scratch of at least fa_bwd_workspace_size(B, H, N, d) bytes, 16-byte
+ *                  aligned, owned by the caller, not used concurrently by another call.
+ * The dQ sum over key blocks runs in a fixed order, so repeated calls on the same inputs
+ * give bitwise identical dq, dk, dv.
+ */
+FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                 const float* lse, void* dq, void* dk, void* dv,
+                 int B, int H, int N, int d, float scale, int causal, const int* seqlens,
+                 void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the calling device's error flag.
+ * Returns FA_OK, FA_ERR_INVALID_ARG (a sequence length outside [1, N] was seen),
+ * FA_ERR_TIMEOUT (a device-side wait gave up; the outputs of that call are undefined) or
+ * FA_ERR_CUDA (the synchronisation itself failed).
+ */
+FA_API fa_status fa_check_device_error(fa_stream_t stream);
+
+/*
+ * Upper bound, in nanoseconds, on every wait inside the kernels (pipeline barriers and the
+ * ordered dQ reduction).  When a wait exceeds it, the kernel records FA_ERR_TIMEOUT, stops
+ * its work and exits instead of hanging.  Default 4e9 (4 s); values below 1e6 are raised to
+ * 1e6.  Applies to launches made after the call, on every device.
+ */
+FA_API void fa_set_wait_timeout_ns(uint64_t ns);
+
+/* Static, human-readable name of a status code. */
+FA_API const char* fa_status_string(fa_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H */

@@ -1,0 +1,159 @@
+"""Exact fused attention for NVIDIA B200 (sm_100a): Python binding of ``include/fa.h``.
+
+This module only marshals arguments: it checks tensor shapes, dtypes and devices, takes raw
+device pointers and the current CUDA stream from PyTorch, and calls the C ABI in
+``libfa.so`` through ctypes.  Every step of the computation runs in the library's CUDA
+kernels; there is no CPU or PyTorch fallback.  If the library is missing or fails to load,
+importing this module raises ``ImportError``.
+
+Build the library with ``python -m io_aware_exact_16_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m io_aware_exact_16_b200.build`")
+try:
+    _lib = ctypes.CDLL(LIB_PATH)
+except OSError as exc:  # pragma: no cover
+    raise ImportError(f"cannot load {LIB_PATH}: {exc}") from exc
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_lib.fa_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, ctypes.c_float, _i, _vp, _vp]
+_lib.fa_fwd.restype = _i
+_lib.fa_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                        ctypes.c_float, _i, _vp, _vp, ctypes.c_size_t, _vp]
+_lib.fa_bwd.restype = _i
+_lib.fa_bwd_workspace_size.argtypes = [_i, _i, _i, _i]
+_lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
+_lib.fa_check_device_error.argtypes = [_vp]
+_lib.fa_check_device_error.restype = _i
+_lib.fa_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+_lib.fa_set_wait_timeout_ns.restype = None
+_lib.fa_status_string.argtypes = [_i]
+_lib.fa_status_string.restype = ctypes.c_char_p
+
+# Every symbol include/fa.h declares.
+EXPORTED = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_check_device_error",
+            "fa_set_wait_timeout_ns", "fa_status_string")
+
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_WORKSPACE = range(6)
+
+
+class FAError(RuntimeError):
+    """A non-FA_OK status from the library."""
+
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+def status_string(status: int) -> str:
+    return _lib.fa_status_string(int(status)).decode()
+
+
+def _stream_handle(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _check_qkv(name: str, t: torch.Tensor, shape, device) -> None:
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _seqlens_ptr(seqlens: Optional[torch.Tensor], B: int, device) -> int:
+    if seqlens is None:
+        return 0
+    if seqlens.dtype != torch.int32 or seqlens.device != device or tuple(seqlens.shape) != (B,):
+        raise ValueError("seqlens must be an int32 tensor of shape [B] on the inputs' device")
+    if not seqlens.is_contiguous():
+        raise ValueError("seqlens must be contiguous")
+    return seqlens.data_ptr()
+
+
+def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+            seqlens: Optional[torch.Tensor] = None, scale: Optional[float] = None,
+            out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None):
+    """``fa_fwd``: returns (O bf16 [B, H, N, d], lse fp32 [B, H, N]) on q's device/stream."""
+    B, H, N, d = q.shape
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_qkv(name, t, (B, H, N, d), dev)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check_qkv("out", out, (B, H, N, d), dev)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    elif lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 tensor [B, H, N]")
+    sc = float(scale) if scale is not None else 1.0 / (d ** 0.5)
+    st = _lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                     B, H, N, d, sc, int(bool(causal)), _seqlens_ptr(seqlens, B, dev),
+                     _stream_handle(dev))
+    if st != FA_OK:
+        raise FAError(st, "fa_fwd")
+    return out, lse
+
+
+def bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(_lib.fa_bwd_workspace_size(B, H, N, d))
+
+
+def backward(q, k, v, o, do, lse, causal: bool = False, seqlens: Optional[torch.Tensor] = None,
+             scale: Optional[float] = None, dq=None, dk=None, dv=None,
+             workspace: Optional[torch.Tensor] = None):
+    """``fa_bwd``: returns (dQ, dK, dV), bf16 [B, H, N, d]."""
+    B, H, N, d = q.shape
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
+        _check_qkv(name, t, (B, H, N, d), dev)
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 tensor [B, H, N]")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _check_qkv(name, t, (B, H, N, d), dev)
+    need = bwd_workspace_size(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    sc = float(scale) if scale is not None else 1.0 / (d ** 0.5)
+    st = _lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                     lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, sc,
+                     int(bool(causal)), _seqlens_ptr(seqlens, B, dev), workspace.data_ptr(),
+                     workspace.numel() * workspace.element_size(), _stream_handle(dev))
+    if st != FA_OK:
+        raise FAError(st, "fa_bwd")
+    return dq, dk, dv
+
+
+def check_device_error(device: Optional[torch.device] = None) -> int:
+    """``fa_check_device_error`` on the current stream; returns the status code."""
+    dev = device or torch.device("cuda", torch.cuda.current_device())
+    with torch.cuda.device(dev):
+        return int(_lib.fa_check_device_error(_stream_handle(dev)))
+
+
+def set_wait_timeout_ns(ns: int) -> None:
+    _lib.fa_set_wait_timeout_ns(int(ns))
+
+
+def raw_library() -> ctypes.CDLL:
+    """The loaded ctypes handle of ``libfa.so`` (for direct C-ABI calls)."""
+    return _lib

@@ -1,0 +1,260 @@
+// fa_api.cu -- host side of the C ABI declared in include/fa.h: argument validation, tensor
+// maps, the per-device error flag and kernel launches.  No compute happens here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <mutex>
+
+#include "fa_internal.h"
+
+namespace fa {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+std::atomic<uint64_t> g_timeout_ns{4000000000ull};
+
+struct DeviceState {
+    bool probed = false;
+    bool supported = false;
+    int num_sms = 0;
+    int* err_flag = nullptr;  // 4-byte device buffer
+};
+DeviceState g_dev[kMaxDevices];
+std::mutex g_mutex;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+EncodeTiledFn encode_fn() {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (g_encode == nullptr) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    return g_encode;
+}
+
+// Returns the current device's state, probing it (and allocating its error flag) once.
+DeviceState* current_device(fa_status* st) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        *st = FA_ERR_CUDA;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceState& s = g_dev[dev];
+    if (!s.probed) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            *st = FA_ERR_CUDA;
+            return nullptr;
+        }
+        s.supported = (major == 10 && minor == 0);
+        s.num_sms = sms;
+        if (s.supported) {
+            if (cudaMalloc(&s.err_flag, sizeof(int)) != cudaSuccess ||
+                cudaMemset(s.err_flag, 0, sizeof(int)) != cudaSuccess) {
+                *st = FA_ERR_CUDA;
+                return nullptr;
+            }
+        }
+        s.probed = true;
+    }
+    if (!s.supported) {
+        *st = FA_ERR_UNSUPPORTED;
+        return nullptr;
+    }
+    *st = FA_OK;
+    return &s;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fa_status check_common(int B, int H, int N, int d, float scale) {
+    if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
+    if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (B > 65535 || H > 65535) return FA_ERR_INVALID_ARG;
+    const long long elems = (long long)B * H * N * d;
+    if (elems >= (1ll << 31)) return FA_ERR_INVALID_ARG;
+    return FA_OK;
+}
+
+int pad128(int N) { return (N + 127) / 128 * 128; }
+
+}  // namespace
+
+bool make_bf16_map(CUtensorMap* map, const void* base, int d, int N, int BH, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_f32_map(CUtensorMap* map, const void* base, int d, int N_pad, int BH, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N_pad, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 4, (cuuint64_t)N_pad * d * 4};
+    cuuint32_t box[3] = {32, (cuuint32_t)box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+const char* fa_status_string(fa_status s) {
+    switch (s) {
+        case FA_OK: return "FA_OK";
+        case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG: invalid argument";
+        case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: unsupported head dim or device";
+        case FA_ERR_CUDA: return "FA_ERR_CUDA: CUDA call failed";
+        case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: a device-side wait timed out";
+        case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    }
+    return "unknown fa_status";
+}
+
+void fa_set_wait_timeout_ns(uint64_t ns) {
+    g_timeout_ns.store(ns < 1000000ull ? 1000000ull : ns);
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int N, int d, float scale, int causal, const int* seqlens, fa_stream_t stream) {
+    fa_status st = check_common(B, H, N, d, scale);
+    if (st != FA_OK) return st;
+    if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return FA_ERR_INVALID_ARG;
+    if (seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u)) return FA_ERR_INVALID_ARG;
+    DeviceState* dev = current_device(&st);
+    if (!dev) return st;
+
+    CUtensorMap tq, tk, tv;
+    if (!make_bf16_map(&tq, q, d, N, B * H, 128) || !make_bf16_map(&tk, k, d, N, B * H, 128) ||
+        !make_bf16_map(&tv, v, d, N, B * H, 128))
+        return FA_ERR_CUDA;
+    FwdParams p{};
+    p.o = o;
+    p.lse = lse;
+    p.seqlens = seqlens;
+    p.err = dev->err_flag;
+    p.H = H;
+    p.N = N;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.causal = causal ? 1 : 0;
+    p.timeout_ns = g_timeout_ns.load();
+    if (launch_fwd(d, tq, tk, tv, p, B, dev->num_sms, reinterpret_cast<cudaStream_t>(stream)) !=
+        cudaSuccess)
+        return FA_ERR_CUDA;
+    return FA_OK;
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+    if (check_common(B, H, N, d, 1.0f) != FA_OK) return 0;
+    const size_t BH = (size_t)B * H;
+    const size_t Np = (size_t)pad128(N);
+    size_t bytes = 0;
+    auto add = [&](size_t n) { bytes += (n + 255) / 256 * 256; };
+    add(BH * N * sizeof(float));           // D
+    add(BH * Np * d * sizeof(float));      // dQ accumulator
+    add(BH * (Np / 128) * sizeof(int));    // ordering counters
+    add(sizeof(int));                      // tile counter
+    return bytes;
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                 const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                 float scale, int causal, const int* seqlens, void* workspace,
+                 size_t workspace_bytes, fa_stream_t stream) {
+    fa_status st = check_common(B, H, N, d, scale);
+    if (st != FA_OK) return st;
+    if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dO) ||
+        !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return FA_ERR_INVALID_ARG;
+    if (seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u)) return FA_ERR_INVALID_ARG;
+    if (!workspace || !aligned16(workspace) || workspace_bytes < fa_bwd_workspace_size(B, H, N, d))
+        return FA_ERR_WORKSPACE;
+    DeviceState* dev = current_device(&st);
+    if (!dev) return st;
+
+    const int BH = B * H;
+    const int Np = pad128(N);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    size_t off = 0;
+    auto take = [&](size_t n) {
+        void* p = ws + off;
+        off += (n + 255) / 256 * 256;
+        return p;
+    };
+    BwdParams p{};
+    p.o = o;
+    p.dO = dO;
+    p.lse = lse;
+    p.dq = dq;
+    p.dk = dk;
+    p.dv = dv;
+    p.Dvec = static_cast<float*>(take((size_t)BH * N * sizeof(float)));
+    p.dq_acc = static_cast<float*>(take((size_t)BH * Np * d * sizeof(float)));
+    p.sem = static_cast<int*>(take((size_t)BH * (Np / 128) * sizeof(int)));
+    p.tile_counter = static_cast<int*>(take(sizeof(int)));
+    p.seqlens = seqlens;
+    p.err = dev->err_flag;
+    p.B = B;
+    p.H = H;
+    p.N = N;
+    p.N_pad = Np;
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.causal = causal ? 1 : 0;
+    p.timeout_ns = g_timeout_ns.load();
+
+    CUtensorMap tq, tk, tv, tdo, tacc;
+    if (!make_bf16_map(&tq, q, d, N, BH, 128) || !make_bf16_map(&tk, k, d, N, BH, 128) ||
+        !make_bf16_map(&tv, v, d, N, BH, 128) || !make_bf16_map(&tdo, dO, d, N, BH, 128) ||
+        !make_f32_map(&tacc, p.dq_acc, d, Np, BH, 128))
+        return FA_ERR_CUDA;
+    if (launch_bwd(d, tq, tk, tv, tdo, tacc, p, dev->num_sms,
+                   reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return FA_ERR_CUDA;
+    return FA_OK;
+}
+
+fa_status fa_check_device_error(fa_stream_t stream) {
+    fa_status st;
+    DeviceState* dev = current_device(&st);
+    if (!dev) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return FA_ERR_CUDA;
+    int flag = 0;
+    if (cudaMemcpy(&flag, dev->err_flag, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return FA_ERR_CUDA;
+    if (flag != 0 && cudaMemset(dev->err_flag, 0, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+    return static_cast<fa_status>(flag);
+}
+
+}  // extern "C"

@@ -1,0 +1,399 @@
+// fa_fwd.cu -- fused exact-attention forward kernel for sm_100a.
+//
+// One CTA owns two 128-row query tiles of one (batch, head) and streams that head's keys and
+// values through shared memory in 128-row blocks, never writing the score matrix to device
+// memory (FlashAttention (DE), "Tiling und blockweise Verarbeitung"; "Zusammenfassen von
+// Operationen in einem CUDA-Kernel").  Per key block j and query tile t:
+//
+//   S_t   = Q_t K_j^T                       tcgen05 MMA, fp32 accumulator in tensor memory
+//   m'    = max(m, rowmax(S_t) * c)         c = scale * log2(e)
+//   P_t   = exp2(S_t * c - m')              bf16, written back over S_t in tensor memory
+//   l     = alpha * l + rowsum(P_t)         alpha = exp2(m - m')
+//   O_t   = alpha * O_t + P_t V_j           tcgen05 MMA with A read from tensor memory
+//
+// which is the online softmax of FlashAttention (DE), "Online-Softmax-Berechnung": a running
+// maximum and a running sum of exponentials, rescaled block by block, so that the final
+// O_t / l equals the two-pass softmax exactly (up to rounding).  The rescale of O is skipped
+// while the running maximum has grown by at most 8 (in log2 units): the stale maximum is then
+// used for both l and O, which stays exact because both share it, and keeps every
+// exponential below 2^8.
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax for query tile 0 (thread r owns row r = TMEM lane r)
+//   warps 4-7  softmax for query tile 1
+//   warp  8    MMA issue (one thread) + TMEM allocation
+//   warp  9    TMA producer (one thread)
+// Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+d) O1 [256+d,256+2d).
+// Shared memory: Q0, Q1, and a ring of K and V blocks, all 128-byte swizzled by TMA.
+#include "fa_internal.h"
+#include "sm100.cuh"
+
+namespace fa {
+namespace {
+
+using namespace sm100;
+
+template <int D>
+struct FwdCfg {
+    static constexpr int BM = 128;                 // query rows per tile
+    static constexpr int BN = 128;                 // keys per block
+    static constexpr int TILES = 2;                // query tiles per CTA
+    static constexpr int ROWS_PER_CTA = BM * TILES;
+    static constexpr int KCH = D / 64;             // 64-column (128-byte) chunks per row
+    static constexpr int STAGES = (D == 128) ? 2 : 3;
+    static constexpr int Q_TILE_BYTES = BM * D * 2;
+    static constexpr int KV_TILE_BYTES = BN * D * 2;
+    static constexpr int CHUNK_BYTES = 128 * 128;  // one 64-column chunk of a 128-row tile
+    static constexpr int SMEM_Q = 0;
+    static constexpr int SMEM_K = SMEM_Q + TILES * Q_TILE_BYTES;
+    static constexpr int SMEM_V = SMEM_K + STAGES * KV_TILE_BYTES;
+    static constexpr int SMEM_BAR = SMEM_V + STAGES * KV_TILE_BYTES;
+    static constexpr int NUM_BARS = 1 + 4 * STAGES + 2 + 2 + 2;
+    static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
+    static constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;  // + alignment slack
+    static constexpr int THREADS = 320;
+    static constexpr uint32_t TMEM_COLS = 512;
+    // tensor-memory column of S_t / O_t for query tile t
+    __device__ static constexpr uint32_t tm_s(int t) { return t ? 128u : 0u; }
+    __device__ static constexpr uint32_t tm_o(int t) { return t ? 256u + D : 256u; }
+};
+
+__device__ __forceinline__ void record_error(int* err, int code) {
+    if (err) atomicCAS(err, 0, code);
+}
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+    using C = FwdCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    const int cta_x = gridDim.x - 1 - blockIdx.x;  // heaviest (causal) query tiles first
+    const int h = blockIdx.y;
+    const int b = blockIdx.z;
+    const int bh = b * p.H + h;
+    const int q_base = cta_x * C::ROWS_PER_CTA;
+
+    int L = p.N;
+    if (p.seqlens != nullptr) {
+        L = p.seqlens[b];
+        if (L < 1 || L > p.N) {
+            if (threadIdx.x == 0) record_error(p.err, kErrInvalidArg);
+            L = L < 1 ? 1 : p.N;
+        }
+    }
+    // Key blocks each query tile needs: keys j < lim, lim = min(L, last row + 1) if causal.
+    auto blocks_for = [&](int row_end) {
+        const int lim = p.causal ? min(L, row_end) : L;
+        return (lim + C::BN - 1) / C::BN;
+    };
+    const int nblk0 = blocks_for(q_base + C::BM);
+    const int nblk1 = blocks_for(q_base + 2 * C::BM);
+
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_BAR);
+    uint64_t* bar_q = bars;
+    uint64_t* bar_kfull = bars + 1;
+    uint64_t* bar_kempty = bar_kfull + C::STAGES;
+    uint64_t* bar_vfull = bar_kempty + C::STAGES;
+    uint64_t* bar_vempty = bar_vfull + C::STAGES;
+    uint64_t* bar_sfull = bar_vempty + C::STAGES;  // [2]
+    uint64_t* bar_pfull = bar_sfull + 2;            // [2]
+    uint64_t* bar_ofull = bar_pfull + 2;            // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SMEM_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::SMEM_MISC + 4);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_q, 1);
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&bar_kfull[s], 1);
+            mbar_init(&bar_kempty[s], 1);
+            mbar_init(&bar_vfull[s], 1);
+            mbar_init(&bar_vempty[s], 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&bar_sfull[t], 1);
+            mbar_init(&bar_pfull[t], C::BM);
+            mbar_init(&bar_ofull[t], 1);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 8) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    auto fail = [&]() {
+        record_error(p.err, kErrTimeout);
+        *abort_flag = 1;
+    };
+
+    if (warp == 9) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_tensormap(&tmQ);
+            prefetch_tensormap(&tmK);
+            prefetch_tensormap(&tmV);
+            mbar_arrive_expect_tx(bar_q, C::TILES * C::Q_TILE_BYTES);
+            for (int t = 0; t < C::TILES; ++t)
+                for (int c = 0; c < C::KCH; ++c)
+                    tma_load_3d(smem + C::SMEM_Q + t * C::Q_TILE_BYTES + c * C::CHUNK_BYTES, &tmQ,
+                                bar_q, c * 64, q_base + t * C::BM, bh);
+            const int n = nblk1;
+            for (int j = 0; j < n; ++j) {
+                const int s = j % C::STAGES;
+                const uint32_t ph = (j / C::STAGES) & 1;
+                if (!mbar_wait(&bar_kempty[s], ph ^ 1, p.timeout_ns, abort_flag)) { fail(); break; }
+                mbar_arrive_expect_tx(&bar_kfull[s], C::KV_TILE_BYTES);
+                for (int c = 0; c < C::KCH; ++c)
+                    tma_load_3d(smem + C::SMEM_K + s * C::KV_TILE_BYTES + c * C::CHUNK_BYTES, &tmK,
+                                &bar_kfull[s], c * 64, j * C::BN, bh);
+                if (!mbar_wait(&bar_vempty[s], ph ^ 1, p.timeout_ns, abort_flag)) { fail(); break; }
+                mbar_arrive_expect_tx(&bar_vfull[s], C::KV_TILE_BYTES);
+                for (int c = 0; c < C::KCH; ++c)
+                    tma_load_3d(smem + C::SMEM_V + s * C::KV_TILE_BYTES + c * C::CHUNK_BYTES, &tmV,
+                                &bar_vfull[s], c * 64, j * C::BN, bh);
+            }
+            // Do not leave the CTA while our copies may still be landing in shared memory.
+            for (int j = max(0, n - C::STAGES); j < n; ++j) {
+                const int s = j % C::STAGES;
+                const uint32_t ph = (j / C::STAGES) & 1;
+                mbar_wait(&bar_kfull[s], ph, p.timeout_ns, abort_flag);
+                mbar_wait(&bar_vfull[s], ph, p.timeout_ns, abort_flag);
+            }
+            if (!mbar_wait(bar_q, 0, p.timeout_ns, abort_flag)) fail();
+        }
+    } else if (warp == 8) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idS = idesc_bf16(C::BM, C::BN, false, false);
+            constexpr uint32_t idPV = idesc_bf16(C::BM, D, false, true);
+            const uint32_t sQ = smem_u32(smem + C::SMEM_Q);
+            const uint32_t sK = smem_u32(smem + C::SMEM_K);
+            const uint32_t sV = smem_u32(smem + C::SMEM_V);
+            const int n0 = nblk0, n1 = nblk1;
+
+            // S_t = Q_t K^T: both operands K-major; 16-column K steps walk the swizzled rows
+            // (32 bytes per step) and then the next 64-column chunk.
+            auto issue_S = [&](int t, int s) {
+                const uint32_t qa = sQ + t * C::Q_TILE_BYTES;
+                const uint32_t ka = sK + s * C::KV_TILE_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk / 4) * C::CHUNK_BYTES + (kk % 4) * 32;
+                    mma_ss(tmem + C::tm_s(t), sdesc_sw128(qa + off, 16, 1024),
+                           sdesc_sw128(ka + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+                }
+            };
+            // O_t += P_t V: P from tensor memory (2 bf16 per column, 8 columns per K step of
+            // 16 keys), V MN-major in shared memory (16 key rows = 2048 bytes per K step; the
+            // two 64-column chunks of d are CHUNK_BYTES apart).
+            auto issue_PV = [&](int t, int s, bool accumulate) {
+                const uint32_t va = sV + s * C::KV_TILE_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < C::BN / 16; ++kk) {
+                    mma_ts(tmem + C::tm_o(t), tmem + C::tm_s(t) + kk * 8,
+                           sdesc_sw128(va + kk * 2048, C::CHUNK_BYTES, 1024), idPV,
+                           (accumulate || kk > 0) ? 1u : 0u);
+                }
+            };
+
+            bool ok = mbar_wait(bar_q, 0, p.timeout_ns, abort_flag);
+            if (ok) ok = mbar_wait(&bar_kfull[0], 0, p.timeout_ns, abort_flag);
+            if (ok) {
+                tc_fence_after();
+                issue_S(0, 0);
+                tc_commit(&bar_sfull[0]);
+                issue_S(1, 0);
+                tc_commit(&bar_sfull[1]);
+                tc_commit(&bar_kempty[0]);
+            }
+            for (int j = 0; ok && j < n1; ++j) {
+                const int s = j % C::STAGES;
+                const uint32_t ph = (j / C::STAGES) & 1;
+                const int jn = j + 1;
+                const int sn = jn % C::STAGES;
+                const uint32_t phn = (jn / C::STAGES) & 1;
+                if (!(ok = mbar_wait(&bar_vfull[s], ph, p.timeout_ns, abort_flag))) break;
+                if (j < n0) {
+                    if (!(ok = mbar_wait(&bar_pfull[0], j & 1, p.timeout_ns, abort_flag))) break;
+                    tc_fence_after();
+                    issue_PV(0, s, j > 0);
+                    tc_commit(&bar_ofull[0]);
+                }
+                if (jn < n1) {
+                    if (!(ok = mbar_wait(&bar_kfull[sn], phn, p.timeout_ns, abort_flag))) break;
+                    tc_fence_after();
+                    if (jn < n0) {
+                        issue_S(0, sn);
+                        tc_commit(&bar_sfull[0]);
+                    }
+                }
+                if (!(ok = mbar_wait(&bar_pfull[1], j & 1, p.timeout_ns, abort_flag))) break;
+                tc_fence_after();
+                issue_PV(1, s, j > 0);
+                tc_commit(&bar_ofull[1]);
+                tc_commit(&bar_vempty[s]);
+                if (jn < n1) {
+                    issue_S(1, sn);
+                    tc_commit(&bar_sfull[1]);
+                    tc_commit(&bar_kempty[sn]);
+                }
+            }
+            if (!ok) fail();
+        }
+    } else {
+        // ------------------------------------------------------------ softmax warpgroups
+        const int t = warp / 4;
+        const int r = threadIdx.x % C::BM;
+        const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
+        const uint32_t tS = tmem + lane_base + C::tm_s(t);
+        const uint32_t tO = tmem + lane_base + C::tm_o(t);
+        const int nt = t ? nblk1 : nblk0;
+        const int row = q_base + t * C::BM + r;
+        const int lim = p.causal ? min(L, row + 1) : L;  // visible keys: j < lim
+        const float c = p.scale_log2;
+        float m = -INFINITY;  // running max of S * c (log2 units), possibly stale by <= 8
+        float l = 0.f;        // running sum of exp2(S * c - m)
+        bool ok = true;
+
+        for (int j = 0; j < nt; ++j) {
+            ok = mbar_wait(&bar_sfull[t], j & 1, p.timeout_ns, abort_flag);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t s[C::BN];
+#pragma unroll
+            for (int q = 0; q < C::BN / 32; ++q) tmem_ld32(tS + q * 32, s + q * 32);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < C::BN / 32; ++q) reg_fence32(s + q * 32);
+
+            const int k0 = j * C::BN;
+            if (k0 + C::BN > lim) {
+#pragma unroll
+                for (int i = 0; i < C::BN; ++i)
+                    if (k0 + i >= lim) s[i] = __float_as_uint(-INFINITY);
+            }
+            float mx = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < C::BN; ++i) mx = fmaxf(mx, __uint_as_float(s[i]));
+            const float m_new = fmaxf(m, mx * c);
+            const bool grow = m_new > m + 8.0f;  // false while both are -inf
+            if (__any_sync(0xffffffffu, grow && j > 0)) {
+                // Rescale this warp's rows of O (alpha = 1 for rows that keep their max).
+                const float alpha = (grow && m != -INFINITY) ? ex2(m - m_new) : 1.0f;
+                ok = mbar_wait(&bar_ofull[t], (j - 1) & 1, p.timeout_ns, abort_flag);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int q = 0; q < D / 32; ++q) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + q * 32, o);
+                    tmem_ld_wait();
+                    reg_fence32(o);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    tmem_st32(tO + q * 32, o);
+                }
+                if (grow) l *= alpha;
+            }
+            if (grow) m = m_new;
+            const float mb = (m == -INFINITY) ? 0.f : m;
+            float rowsum = 0.f;
+            uint32_t pk[C::BN / 2];
+#pragma unroll
+            for (int i = 0; i < C::BN / 2; ++i) {
+                const float p0 = ex2(fmaf(__uint_as_float(s[2 * i]), c, -mb));
+                const float p1 = ex2(fmaf(__uint_as_float(s[2 * i + 1]), c, -mb));
+                rowsum += p0 + p1;
+                pk[i] = pack_bf16x2(p0, p1);
+            }
+            l += rowsum;
+#pragma unroll
+            for (int q = 0; q < C::BN / 64; ++q) tmem_st32(tS + q * 32, pk + q * 32);
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&bar_pfull[t]);
+        }
+
+        // ------------------------------------------------------------ epilogue
+        if (ok) ok = mbar_wait(&bar_ofull[t], (nt - 1) & 1, p.timeout_ns, abort_flag);
+        if (__all_sync(0xffffffffu, ok)) {
+            tc_fence_after();
+            const float inv_l = l > 0.f ? 1.0f / l : 0.f;
+            const bool in_range = row < p.N;
+            __nv_bfloat16* orow =
+                reinterpret_cast<__nv_bfloat16*>(p.o) + ((size_t)bh * p.N + (in_range ? row : 0)) * D;
+#pragma unroll
+            for (int q = 0; q < D / 32; ++q) {
+                uint32_t o[32];
+                tmem_ld32(tO + q * 32, o);
+                tmem_ld_wait();
+                reg_fence32(o);
+                uint32_t w[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l,
+                                       __uint_as_float(o[2 * i + 1]) * inv_l);
+                if (in_range) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                }
+            }
+            if (in_range) {
+                // lse in natural-log units: (m + log2 l) * ln 2
+                p.lse[(size_t)bh * p.N + row] =
+                    l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+            }
+        } else {
+            fail();
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 8) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+template <int D>
+cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                         const FwdParams& p, int B, cudaStream_t stream) {
+    using C = FwdCfg<D>;
+    static bool configured = false;  // attribute set once per process (idempotent if raced)
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(fa_fwd_kernel<D>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    dim3 grid((p.N + C::ROWS_PER_CTA - 1) / C::ROWS_PER_CTA, p.H, B);
+    fa_fwd_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const FwdParams& p, int B, int num_sms, cudaStream_t stream) {
+    (void)num_sms;
+    if (d == 64) return launch_fwd_d<64>(tq, tk, tv, p, B, stream);
+    return launch_fwd_d<128>(tq, tk, tv, p, B, stream);
+}
+
+}  // namespace fa

@@ -1,0 +1,61 @@
+// fa_internal.h -- declarations shared by the host ABI (fa_api.cu) and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/fa.h"
+
+namespace fa {
+
+// Device error-flag codes mirror fa_status.
+constexpr int kErrInvalidArg = FA_ERR_INVALID_ARG;
+constexpr int kErrTimeout = FA_ERR_TIMEOUT;
+
+struct FwdParams {
+    void* o;               // bf16 [B, H, N, d]
+    float* lse;            // fp32 [B, H, N]
+    const int* seqlens;    // device int32 [B] or nullptr
+    int* err;              // device error flag
+    int H, N;
+    float scale_log2;      // scale * log2(e)
+    int causal;
+    uint64_t timeout_ns;
+};
+
+struct BwdParams {
+    const void* o;         // bf16 [B, H, N, d]
+    const void* dO;        // bf16 [B, H, N, d]
+    const float* lse;      // fp32 [B, H, N]
+    void* dq;              // bf16 out
+    void* dk;              // bf16 out
+    void* dv;              // bf16 out
+    float* Dvec;           // fp32 [B, H, N]   workspace
+    float* dq_acc;         // fp32 [B, H, N_pad, d] workspace
+    int* sem;              // int32 [B, H, N_pad / 128] workspace (ordered-reduction counters)
+    int* tile_counter;     // int32 [1] workspace
+    const int* seqlens;
+    int* err;
+    int B, H, N, N_pad;
+    float scale;
+    float scale_log2;
+    int causal;
+    uint64_t timeout_ns;
+};
+
+// Tensor maps: a bf16 [B*H, N, d] tensor seen as 3-D (d, N, B*H), 128-byte swizzle,
+// box = 64 columns x `box_rows` rows; rows past N read as zeros.
+bool make_bf16_map(CUtensorMap* map, const void* base, int d, int N, int BH, int box_rows);
+// An fp32 [B*H, N_pad, d] tensor seen as 3-D (d, N_pad, B*H), 128-byte swizzle,
+// box = 32 columns x `box_rows` rows.
+bool make_f32_map(CUtensorMap* map, const void* base, int d, int N_pad, int BH, int box_rows);
+
+cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const FwdParams& p, int B, int num_sms, cudaStream_t stream);
+
+cudaError_t launch_bwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tdo, const CUtensorMap& tdq_acc, const BwdParams& p,
+                       int num_sms, cudaStream_t stream);
+
+}  // namespace fa
