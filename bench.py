@@ -1,0 +1,413 @@
+"""Benchmark: bf16 exact-attention forward + backward TFLOP/s on B200.
+
+One step = one pass of the whole hot path over one batch: ``fa_fwd`` (fused forward) then
+``fa_bwd`` (preprocess, fused backward, dQ convert) on the same seeded synthetic inputs.
+Default workload: the throughput-sweep shape at N = 4096, H = 16, d = 128, non-causal,
+B = 16384 / N = 4 per GPU (the size at which the throughput targets are stated).
+
+FLOP accounting: forward 4*B*H*N^2*d (halved when causal), backward 2.5x the forward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+With N > 1 launch one process per GPU with torch.distributed.run; each rank runs its own
+batch of the same shape (weak scaling, no collective on the data path) and rank 0 prints one
+JSON line with the time taken as the maximum over ranks.
+
+``--impl reference`` times the fp64 CPU oracle (the plain definition of attention) on a bounded
+sample of the same workload; it is a deliberately slow reference, not a target.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "bf16 attention fwd/bwd TFLOP/s and % of B200 dense BF16 tensor peak"
+NOMINAL_PEAK_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+WORKLOADS = {
+    "sweep-N4096-H16-d128": lambda: workloads.sweep(4096, 16, 128, False),
+    "sweep-N4096-H16-d128-causal": lambda: workloads.sweep(4096, 16, 128, True),
+    "sweep-N16384-H16-d128": lambda: workloads.sweep(16384, 16, 128, False),
+    "sweep-N4096-H32-d64": lambda: workloads.sweep(4096, 32, 64, False),
+    "gpt2-small": workloads.gpt2_small,
+    "bert-large-padded": workloads.bert_large_padded,
+}
+DEFAULT_WORKLOAD = "sweep-N4096-H16-d128"
+
+
+def flops_per_step(w: workloads.Workload, seqlens=None) -> tuple[float, float]:
+    """(forward, backward) algorithmic FLOPs for one batch; padded keys count as skipped work."""
+    if seqlens is not None:
+        keys = float(sum(int(x) for x in seqlens))  # effective: sum_b L_b instead of B*N
+        fwd = 4.0 * w.H * w.N * keys * w.d
+    else:
+        fwd = 4.0 * w.B * w.H * w.N * w.N * w.d
+    if w.causal:
+        fwd /= 2.0
+    return fwd, 2.5 * fwd
+
+
+def load_peaks() -> tuple[dict, str]:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("fa_bwd.cu", "fa_fwd.cu", "sm100.cuh", "fa_internal.h"):
+        with open(os.path.join(ROOT, "io_aware_exact_16_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def dram_traffic(kernel: str, workload: str) -> float | None:
+    """Per-launch DRAM bytes from the committed ncu summary, or None when it is stale."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            data = json.load(f)
+    except (OSError, ValueError):
+        return None
+    entry = data.get(kernel, {})
+    if entry.get("workload") != workload or entry.get("source_hash") != kernel_source_hash():
+        return None
+    return float(entry["dram_bytes_per_launch"])
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.out = None
+
+    def __enter__(self):
+        try:
+            self.out = open(f"/tmp/fa_bench_clocks_{os.getpid()}.csv", "w", buffering=1)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+            return self
+        # wait (up to 3 s) for the first sample so the timed region is covered
+        t0 = time.time()
+        while time.time() - t0 < 3.0 and self.proc.poll() is None:
+            try:
+                if os.path.getsize(self.out.name) > 0:
+                    break
+            except OSError:
+                break
+            time.sleep(0.05)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.out is not None:
+            self.out.close()
+
+    def summary(self) -> dict | None:
+        if self.proc is None or self.out is None:
+            return None
+        try:
+            with open(self.out.name) as f:
+                lines = [l.strip() for l in f if l.strip()]
+            os.unlink(self.out.name)
+        except OSError:
+            return None
+        sms, maxes, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sms.append(float(parts[1]))
+                maxes.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sms:
+            return None
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxes),
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
+    import io_aware_exact_16_b200 as fa
+
+    w = WORKLOADS[args.workload]()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    # Each rank draws its own batch (seed offset by rank): weak scaling over independent batches.
+    w_rank = workloads.Workload(w.name, w.B, w.H, w.N, w.d, w.causal, w.seed + 7919 * rank,
+                                w.std, w.pad_range)
+    inp = workloads.make_inputs(w_rank)
+    sl_cpu = inp.seqlens
+    fwd_flops, bwd_flops = flops_per_step(w, sl_cpu)
+    step_flops = fwd_flops + bwd_flops
+
+    pinned = {n: getattr(inp, n).pin_memory() for n in ("q", "k", "v", "do")}
+    q, k, v, do = (pinned[n].to(dev, non_blocking=True) for n in ("q", "k", "v", "do"))
+    sl = sl_cpu.to(dev) if sl_cpu is not None else None
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.bwd_workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        fa.forward(q, k, v, causal=w.causal, seqlens=sl, scale=w.scale, out=o, lse=lse)
+        fa.backward(q, k, v, o, do, lse, causal=w.causal, seqlens=sl, scale=w.scale,
+                    dq=dq, dk=dk, dv=dv, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if fa.check_device_error(dev) != 0:
+        raise RuntimeError("device error flag set during warm-up")
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    # ---- timed region: per-pass CUDA events on the launching stream
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clocks:
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for s in range(args.steps):
+            ev[s][0].record(stream)
+            fa.forward(q, k, v, causal=w.causal, seqlens=sl, scale=w.scale, out=o, lse=lse)
+            ev[s][1].record(stream)
+            fa.backward(q, k, v, o, do, lse, causal=w.causal, seqlens=sl, scale=w.scale,
+                        dq=dq, dk=dk, dv=dv, workspace=ws)
+            ev[s][2].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    elapsed_ms = start.elapsed_time(end)
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    status = fa.check_device_error(dev)
+    if status != 0:
+        raise RuntimeError(f"device error flag {status} after the timed region")
+
+    # ---- end-to-end through the public API: pinned host inputs in, host results out
+    host_out = {n: torch.empty_like(pinned["q"]).pin_memory() for n in ("o", "dq", "dk", "dv")}
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    e2e_steps = max(1, min(args.steps, 5))
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for n, t in (("q", q), ("k", k), ("v", v), ("do", do)):
+            t.copy_(pinned[n], non_blocking=True)
+        step()
+        for n, t in (("o", o), ("dq", dq), ("dk", dk), ("dv", dv)):
+            host_out[n].copy_(t, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+
+    times = torch.tensor([elapsed_ms, e2e_ms, fwd_ms, bwd_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
+    elapsed_ms, e2e_ms, fwd_ms, bwd_ms = times.tolist()
+    if rank != 0:
+        return None
+
+    peaks, peak_src = load_peaks()
+    sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    value = step_flops * args.steps * world / (elapsed_ms * 1e-3) / 1e12
+    ms_per_step = elapsed_ms / args.steps
+    bwd_tflops = bwd_flops / (bwd_ms * 1e-3) / 1e12
+    fwd_tflops = fwd_flops / (fwd_ms * 1e-3) / 1e12
+    wname = args.workload
+    traffic = dram_traffic("fa_bwd_kernel", wname)
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) draws rounded to bf16)",
+        "pct_of_dense_bf16_peak": round(100.0 * value / world / NOMINAL_PEAK_TFLOPS, 2),
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                   "causal": w.causal, "padded": w.pad_range is not None,
+                   "per_gpu_batch": w.B, "global_batch": w.B * world,
+                   "parallelism": f"independent batches x{world}",
+                   "l2": "inputs larger than L2: Q,K,V,O,dO,dQ,dK,dV are %.0f MB each per GPU"
+                         % (w.B * w.H * w.N * w.d * 2 / 1e6)},
+        "passes": {"fwd_ms": round(fwd_ms, 4), "bwd_ms": round(bwd_ms, 4),
+                   "fwd_tflops": round(fwd_tflops, 2), "bwd_tflops": round(bwd_tflops, 2),
+                   "fwd_pct_of_2250": round(100 * fwd_tflops / NOMINAL_PEAK_TFLOPS, 2),
+                   "bwd_pct_of_2250": round(100 * bwd_tflops / NOMINAL_PEAK_TFLOPS, 2)},
+        "roofline": {
+            "kernel": "fa_bwd (preprocess + fused backward + dQ convert; the fused backward "
+                      "kernel is ~95% of the pass)",
+            "bound": "tensor", "achieved": round(bwd_tflops, 2),
+            "peak": sustained, "unit": "TFLOP/s",
+            "frac": round(bwd_tflops / sustained, 4),
+            "peak_source": f"{peak_src} bf16 sustained (MEASURED_PEAKS.json)",
+            "traffic": traffic,
+        },
+        "roofline_fwd": {
+            "kernel": "fa_fwd_kernel", "bound": "tensor", "achieved": round(fwd_tflops, 2),
+            "peak": sustained, "unit": "TFLOP/s", "frac": round(fwd_tflops / sustained, 4),
+            "traffic": dram_traffic("fa_fwd_kernel", wname),
+        },
+        "e2e": {"value": round(step_flops * e2e_steps * world / (e2e_ms * 1e-3) / 1e12, 2),
+                "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_heads)
+    return line
+
+
+def cpu_baseline(w: workloads.Workload, inp, heads: int) -> dict:
+    """The oracle as it stands, fwd + bwd on a bounded sample of heads of the same workload."""
+    import oracle
+
+    oracle.build()
+    total = w.B * w.H
+    picks = workloads.seeded_sample(w.seed + 99, total, heads)
+    t0 = time.perf_counter()
+    flops = 0.0
+    for flat in picks:
+        b, h = divmod(flat, w.H)
+        L = int(inp.seqlens[b]) if inp.seqlens is not None else w.N
+        oracle.head_bwd(inp.q[b, h], inp.k[b, h], inp.v[b, h], inp.do[b, h], w.scale, w.causal, L)
+        f = 4.0 * w.N * L * w.d * (0.5 if w.causal else 1.0)
+        flops += 3.5 * f
+    dt = time.perf_counter() - t0
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.get_threads(),
+            "kind": "oracle",
+            "sample": f"fp64 C oracle fwd+bwd on {len(picks)} of {total} heads ({dt:.1f} s)"}
+
+
+def run_reference(args, rank: int, world: int) -> dict | None:
+    if rank != 0:
+        return None
+    import oracle
+
+    oracle.build()
+    w = WORKLOADS[args.workload]()
+    inp = workloads.make_inputs(w)
+    fwd_flops, bwd_flops = flops_per_step(w, inp.seqlens)
+    head_flops = (fwd_flops + bwd_flops) / (w.B * w.H)  # one head per step (bounded sample)
+    heads = workloads.seeded_sample(w.seed + 99, w.B * w.H, args.warmup + args.steps)
+
+    def one(flat):
+        b, h = divmod(flat, w.H)
+        L = int(inp.seqlens[b]) if inp.seqlens is not None else w.N
+        oracle.head_bwd(inp.q[b, h], inp.k[b, h], inp.v[b, h], inp.do[b, h], w.scale, w.causal, L)
+
+    for i in range(args.warmup):
+        one(heads[i % len(heads)])
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        one(heads[(args.warmup + i) % len(heads)])
+    dt = time.perf_counter() - t0
+    value = head_flops * args.steps / dt / 1e12
+    return {
+        "impl": "reference",
+        "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt * 1e3 / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.get_threads(),
+                         "kind": "oracle",
+                         "sample": f"one head of {w.B * w.H} per step, fp64 fwd+bwd"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main() -> int:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--cpu-heads", type=int, default=12)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    distributed = world > 1 and args.impl == "ours"
+    if distributed:
+        import datetime
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, rank, world)
+        else:
+            line = run_ours(args, rank, world, local_rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if distributed:
+            torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

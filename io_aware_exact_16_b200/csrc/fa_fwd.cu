@@ -48,7 +48,7 @@ struct FwdCfg {
     static constexpr int SMEM_K = SMEM_Q + TILES * Q_TILE_BYTES;
     static constexpr int SMEM_V = SMEM_K + STAGES * KV_TILE_BYTES;
     static constexpr int SMEM_BAR = SMEM_V + STAGES * KV_TILE_BYTES;
-    static constexpr int NUM_BARS = 1 + 4 * STAGES + 2 + 2 + 2;
+    static constexpr int NUM_BARS = 1 + 4 * STAGES + 2 + 2 + 2 + 1;
     static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;  // + alignment slack
     static constexpr int THREADS = 320;
@@ -104,6 +104,7 @@ __global__ void __launch_bounds__(320, 1)
     uint64_t* bar_sfull = bar_vempty + C::STAGES;  // [2]
     uint64_t* bar_pfull = bar_sfull + 2;            // [2]
     uint64_t* bar_ofull = bar_pfull + 2;            // [2]
+    uint64_t* bar_done = bar_ofull + 2;             // every MMA of this CTA finished
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SMEM_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::SMEM_MISC + 4);
 
@@ -120,6 +121,7 @@ __global__ void __launch_bounds__(320, 1)
             mbar_init(&bar_pfull[t], C::BM);
             mbar_init(&bar_ofull[t], 1);
         }
+        mbar_init(bar_done, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -250,6 +252,9 @@ __global__ void __launch_bounds__(320, 1)
                 }
             }
             if (!ok) fail();
+            // Wait for every MMA issued here before tensor memory can be released.
+            tc_commit(bar_done);
+            mbar_wait(bar_done, 0, p.timeout_ns, abort_flag);
         }
     } else {
         // ------------------------------------------------------------ softmax warpgroups
