@@ -164,6 +164,20 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sms)}
 
 
+def rank_workload(w: workloads.Workload, rank: int) -> workloads.Workload:
+    """The batch rank `rank` processes: same shape, its own seed (independent batches)."""
+    return workloads.Workload(w.name, w.B, w.H, w.N, w.d, w.causal, w.seed + 7919 * rank, w.std,
+                              w.pad_range)
+
+
+def reduce_max(values: list[float], world: int, device=None) -> list[float]:
+    """Element-wise maximum over ranks (the job takes as long as its slowest rank)."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
 def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     import io_aware_exact_16_b200 as fa
 
@@ -171,9 +185,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     # Each rank draws its own batch (seed offset by rank): weak scaling over independent batches.
-    w_rank = workloads.Workload(w.name, w.B, w.H, w.N, w.d, w.causal, w.seed + 7919 * rank,
-                                w.std, w.pad_range)
-    inp = workloads.make_inputs(w_rank)
+    inp = workloads.make_inputs(rank_workload(w, rank))
     sl_cpu = inp.seqlens
     fwd_flops, bwd_flops = flops_per_step(w, sl_cpu)
     step_flops = fwd_flops + bwd_flops
@@ -248,10 +260,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     barrier()
     e2e_ms = e0.elapsed_time(e1)
 
-    times = torch.tensor([elapsed_ms, e2e_ms, fwd_ms, bwd_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
-    elapsed_ms, e2e_ms, fwd_ms, bwd_ms = times.tolist()
+    elapsed_ms, e2e_ms, fwd_ms, bwd_ms = reduce_max([elapsed_ms, e2e_ms, fwd_ms, bwd_ms], world,
+                                                    dev)
     if rank != 0:
         return None
 

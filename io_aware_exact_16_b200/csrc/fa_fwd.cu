@@ -18,11 +18,14 @@
 // used for both l and O, which stays exact because both share it, and keeps every
 // exponential below 2^8.
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads = 3 warpgroups):
 //   warps 0-3  softmax for query tile 0 (thread r owns row r = TMEM lane r)
 //   warps 4-7  softmax for query tile 1
 //   warp  8    MMA issue (one thread) + TMEM allocation
 //   warp  9    TMA producer (one thread)
+//   warps 10-11 idle
+// The third warpgroup hands most of its registers to the two softmax warpgroups
+// (setmaxnreg: 56 + 2 x 224 per thread slot = 3 x 168 launched).
 // Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+d) O1 [256+d,256+2d).
 // Shared memory: Q0, Q1, and a ring of K and V blocks, all 128-byte swizzled by TMA.
 #include "fa_internal.h"
@@ -51,7 +54,8 @@ struct FwdCfg {
     static constexpr int NUM_BARS = 1 + 4 * STAGES + 2 + 2 + 2 + 1;
     static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;  // + alignment slack
-    static constexpr int THREADS = 320;
+    static constexpr int THREADS = 384;
+    static constexpr uint32_t REGS_SOFTMAX = 224, REGS_OTHER = 56;
     static constexpr uint32_t TMEM_COLS = 512;
     // tensor-memory column of S_t / O_t for query tile t
     __device__ static constexpr uint32_t tm_s(int t) { return t ? 128u : 0u; }
@@ -63,7 +67,7 @@ __device__ __forceinline__ void record_error(int* err, int code) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
     using C = FwdCfg<D>;
@@ -139,7 +143,9 @@ __global__ void __launch_bounds__(320, 1)
         *abort_flag = 1;
     };
 
-    if (warp == 9) {
+    if (warp >= 8) {
+      regs_decrease<C::REGS_OTHER>();
+      if (warp == 9) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             prefetch_tensormap(&tmQ);
@@ -256,7 +262,9 @@ __global__ void __launch_bounds__(320, 1)
             tc_commit(bar_done);
             mbar_wait(bar_done, 0, p.timeout_ns, abort_flag);
         }
+      }
     } else {
+        regs_increase<C::REGS_SOFTMAX>();
         // ------------------------------------------------------------ softmax warpgroups
         const int t = warp / 4;
         const int r = threadIdx.x % C::BM;
@@ -288,17 +296,57 @@ __global__ void __launch_bounds__(320, 1)
                 for (int i = 0; i < C::BN; ++i)
                     if (k0 + i >= lim) s[i] = __float_as_uint(-INFINITY);
             }
-            float mx = -INFINITY;
+            // Row maximum as 8 independent chains, then a small tree.
+            float mx8[8];
 #pragma unroll
-            for (int i = 0; i < C::BN; ++i) mx = fmaxf(mx, __uint_as_float(s[i]));
+            for (int k = 0; k < 8; ++k) mx8[k] = __uint_as_float(s[k]);
+#pragma unroll
+            for (int i = 8; i < C::BN; i += 8)
+#pragma unroll
+                for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], __uint_as_float(s[i + k]));
+#pragma unroll
+            for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+                for (int k = 0; k < w; ++k) mx8[k] = fmaxf(mx8[k], mx8[k + w]);
+            const float mx = mx8[0];
             const float m_new = fmaxf(m, mx * c);
             const bool grow = m_new > m + 8.0f;  // false while both are -inf
+            // alpha rescales what was accumulated under the old maximum (1 when it is kept).
+            const float alpha = (grow && m != -INFINITY) ? ex2(m - m_new) : 1.0f;
+            if (grow) {
+                l *= alpha;
+                m = m_new;
+            }
+            const float mb = (m == -INFINITY) ? 0.f : m;
+            // p = exp2(S * c - m): the argument as packed two-wide FMAs, the exponential on the
+            // MUFU unit, the row sum in 4 packed accumulators (8 independent chains).  P goes to
+            // tensor memory in two 64-key halves, over S columns already read.
+            const float2 c2 = make_float2(c, c);
+            const float2 nm2 = make_float2(-mb, -mb);
+            float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                             make_float2(0.f, 0.f)};
+#pragma unroll
+            for (int h = 0; h < C::BN / 64; ++h) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int e0 = h * 64 + 2 * i;
+                    const float2 x = ffma2(make_float2(__uint_as_float(s[e0]),
+                                                       __uint_as_float(s[e0 + 1])), c2, nm2);
+                    const float2 e = make_float2(ex2(x.x), ex2(x.y));
+                    acc[i % 4] = fadd2(acc[i % 4], e);
+                    pk[i] = pack_bf16x2(e.x, e.y);
+                }
+                tmem_st32(tS + h * 32, pk);
+            }
+            l += ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+                 ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
             if (__any_sync(0xffffffffu, grow && j > 0)) {
-                // Rescale this warp's rows of O (alpha = 1 for rows that keep their max).
-                const float alpha = (grow && m != -INFINITY) ? ex2(m - m_new) : 1.0f;
+                // Rescale this warp's rows of O once the previous P V has landed.
                 ok = mbar_wait(&bar_ofull[t], (j - 1) & 1, p.timeout_ns, abort_flag);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 tc_fence_after();
+                const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
                 for (int q = 0; q < D / 32; ++q) {
                     uint32_t o[32];
@@ -306,25 +354,15 @@ __global__ void __launch_bounds__(320, 1)
                     tmem_ld_wait();
                     reg_fence32(o);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    for (int i = 0; i < 32; i += 2) {
+                        const float2 y = fmul2(make_float2(__uint_as_float(o[i]),
+                                                           __uint_as_float(o[i + 1])), a2);
+                        o[i] = __float_as_uint(y.x);
+                        o[i + 1] = __float_as_uint(y.y);
+                    }
                     tmem_st32(tO + q * 32, o);
                 }
-                if (grow) l *= alpha;
             }
-            if (grow) m = m_new;
-            const float mb = (m == -INFINITY) ? 0.f : m;
-            float rowsum = 0.f;
-            uint32_t pk[C::BN / 2];
-#pragma unroll
-            for (int i = 0; i < C::BN / 2; ++i) {
-                const float p0 = ex2(fmaf(__uint_as_float(s[2 * i]), c, -mb));
-                const float p1 = ex2(fmaf(__uint_as_float(s[2 * i + 1]), c, -mb));
-                rowsum += p0 + p1;
-                pk[i] = pack_bf16x2(p0, p1);
-            }
-            l += rowsum;
-#pragma unroll
-            for (int q = 0; q < C::BN / 64; ++q) tmem_st32(tS + q * 32, pk + q * 32);
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&bar_pfull[t]);

@@ -1,0 +1,96 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every symbol that
+include/fa.h declares, and rejects bad arguments before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import io_aware_exact_16_b200 as fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+
+def declared_symbols():
+    with open(HEADER) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"FA_API\s+[\w\s\*]+?\b(fa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_symbols()
+    for n in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_check_device_error",
+              "fa_status_string", "fa_set_wait_timeout_ns"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(fa.LIB_PATH)
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    assert set(declared_symbols()) == set(fa.EXPORTED)
+
+
+def test_status_strings():
+    for code in range(6):
+        assert fa.status_string(code).startswith("FA_")
+    assert "unknown" in fa.status_string(99)
+
+
+def test_workspace_size_formula():
+    # D (fp32 per row) + dQ accumulator (fp32, rows padded to 128) + counters + tile counter,
+    # each rounded up to 256 bytes.
+    def r(n):
+        return (n + 255) // 256 * 256
+    for B, H, N, d in ((1, 1, 1, 64), (2, 3, 300, 128), (4, 16, 4096, 128)):
+        Np = (N + 127) // 128 * 128
+        expect = r(B * H * N * 4) + r(B * H * Np * d * 4) + r(B * H * (Np // 128) * 4) + r(4)
+        assert fa.bwd_workspace_size(B, H, N, d) == expect
+    assert fa.bwd_workspace_size(1, 1, 128, 96) == 0
+    assert fa.bwd_workspace_size(0, 1, 128, 64) == 0
+
+
+def _fwd(lib, *, ptr=16, B=1, H=1, N=8, d=64, scale=0.125, seqlens=None):
+    return lib.fa_fwd(ptr, ptr, ptr, ptr, ptr, B, H, N, d, ctypes.c_float(scale), 0, seqlens, None)
+
+
+def test_forward_rejects_bad_arguments_without_a_device():
+    lib = fa.raw_library()
+    assert _fwd(lib, d=96) == fa.FA_ERR_UNSUPPORTED
+    assert _fwd(lib, N=0) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(lib, B=0) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(lib, scale=0.0) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(lib, scale=float("nan")) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(lib, scale=float("inf")) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(lib, ptr=None) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(lib, ptr=24) == fa.FA_ERR_INVALID_ARG          # not 16-byte aligned
+    assert _fwd(lib, seqlens=18) == fa.FA_ERR_INVALID_ARG      # not 4-byte aligned
+    assert _fwd(lib, B=1 << 16) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(lib, B=2048, H=64, N=4096, d=128) == fa.FA_ERR_INVALID_ARG  # > 2^31 elements
+
+
+def test_backward_rejects_bad_arguments_and_short_workspace_without_a_device():
+    lib = fa.raw_library()
+    need = fa.bwd_workspace_size(1, 1, 8, 64)
+
+    def bwd(ws=16, ws_bytes=need, d=64, ptr=16):
+        return lib.fa_bwd(ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, 1, 1, 8, d,
+                          ctypes.c_float(0.125), 0, None, ws, ws_bytes, None)
+
+    assert bwd(d=80) == fa.FA_ERR_UNSUPPORTED
+    assert bwd(ptr=None) == fa.FA_ERR_INVALID_ARG
+    assert bwd(ws=None) == fa.FA_ERR_WORKSPACE
+    assert bwd(ws_bytes=need - 1) == fa.FA_ERR_WORKSPACE
+    assert bwd(ws=32 + 8) == fa.FA_ERR_WORKSPACE
+
+
+def test_python_binding_checks_shapes_before_calling():
+    import torch
+    q = torch.zeros((1, 1, 8, 64), dtype=torch.float32)
+    with pytest.raises(TypeError):
+        fa.forward(q, q, q)
+    qb = torch.zeros((1, 1, 8, 64), dtype=torch.bfloat16)
+    kb = torch.zeros((1, 1, 9, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fa.forward(qb, kb, qb)
