@@ -231,6 +231,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
     p.scale = scale;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
+    p.resident_ctas = dev->num_sms;
     p.timeout_ns = g_timeout_ns.load();
 
     CUtensorMap tq, tk, tv, tdo, tacc;

@@ -16,16 +16,31 @@
 //                       key-block order (deterministic)
 //   fa_bwd_dq_kernel    dQ = scale * accumulator -> bf16
 //
-// Main-kernel warp roles (320 threads):
-//   warps 0-3  S/dP -> P, dS (thread r owns key row r = TMEM lane r)
-//   warps 4-7  dQ drain (thread r owns query row r) + dK/dV epilogue
-//   warp  8    MMA issue (one thread) + TMEM allocation
-//   warp  9    TMA producer (one thread)
-// Tensor memory (512 columns): A [0,128) S^T -> P^T (bf16) -> dQ block (fp32, d columns)
-//                              B [128,256) dP^T -> dS^T (bf16)
-//                              dV [256, 256+d)   dK [256+d, 256+2d)
+// Main-kernel warp roles (512 threads = 4 warpgroups):
+//   warps 0-7   compute: warpgroup h owns query columns [64h, 64h+64) of every block; thread
+//               (h, r) owns key row r (= TMEM lane r).  Per query block two phases:
+//                 P   (needs S^T)  P^T = exp2(S^T c - lse2)   -> tensor memory (bf16)
+//                 dS  (needs dP^T) dS^T = P^T (dP^T - D)      -> tensor + shared memory (bf16)
+//               each overlapping one MMA (dP^T under P, dV under dS).  At the end they write
+//               dV (warpgroup 0) and dK (warpgroup 1).
+//   warp  8     MMA issue (one thread) + TMEM allocation
+//   warp  9     TMA producer (one thread)
+//   warp  10    ordering of the dQ adds, turns (one thread): waits until it is this key block's
+//               turn to add into query block i and says so (bar_go)
+//   warp  11    ordering of the dQ adds, counts (one thread): once the adds are issued
+//               (bar_added), fences and publishes the new count; a separate thread so that
+//               neither the fence nor this CTA's own adds ever hold up a turn
+//   warps 12-15 dQ drain: copy the dQ block out of tensor memory, free it, add it to the
+//               fp32 accumulator.  For d = 128 the block is held transposed (dQ^T = K^T dS^T,
+//               lane = feature, column = query), so each warp adds whole 128-byte lines; for
+//               d = 64 it is dQ = dS K (lane = query) added with 16-byte vector adds.
+// Registers: warpgroup 2 gives its share to warpgroups 0, 1 and 3 (setmaxnreg).
+// Tensor memory (512 columns):
+//   A [0,128)   S^T (fp32) -> P^T (bf16, columns [0,64))
+//   B [128,256) dP^T (fp32) -> dS^T (bf16, [128,192)) -> the dQ block (fp32)
+//   dV [256, 256+d)   dK [256+d, 256+2d)
 // Shared memory: K_j, V_j (once), a 2-stage ring of Q_i / dO_i, dS^T (bf16, 128-byte
-// swizzled, written by warps 0-3 for the dQ MMA), lse*log2(e) and D of the query block.
+// swizzled, an operand of the dQ MMA), lse*log2(e) and D of the query blocks.
 #include "fa_internal.h"
 #include "sm100.cuh"
 
@@ -53,10 +68,12 @@ struct BwdCfg {
     static constexpr int SMEM_DS = SMEM_DO + QST * Q_TILE_BYTES;
     static constexpr int SMEM_VEC = SMEM_DS + DS_BYTES;       // [2][128] lse2, [2][128] D
     static constexpr int SMEM_BAR = SMEM_VEC + 4 * BM * 4;
-    static constexpr int NUM_BARS = 1 + 2 * QST + 5;
+    static constexpr int NUM_BARS = 1 + 2 * QST + 11;
     static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
-    static constexpr int SMEM_BYTES = SMEM_MISC + 16;
-    static constexpr int THREADS = 320;
+    static constexpr int SMEM_BYTES = SMEM_MISC + 16;  // tmem address, abort, tile, progress
+    static constexpr int THREADS = 512;
+    // 2 x 160 (compute) + 56 (MMA / TMA / ordering) + 136 (drain) = 4 x 128 launched
+    static constexpr uint32_t REGS_COMPUTE = 160, REGS_OTHER = 56, REGS_DRAIN = 136;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t TM_A = 0, TM_B = 128, TM_DV = 256, TM_DK = 256 + D;
 };
@@ -130,8 +147,20 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const BwdParams p, long 
 }
 
 // ---------------------------------------------------------------------------- main kernel
+// Position of key block j in the fixed order in which key blocks add into query block i.
+// Causal: blocks visit i from j upwards, so they reach i in the order j = jmax, jmax-1, ..., 0.
+// Non-causal, rotated: block j visits i = j, j+1, ..., n-1, 0, ..., j-1 and reaches i at step
+// (i - j) mod n, so the order is j = i, i-1, ..., 0, V-1, ..., i+1 (V = key blocks present).
+// Non-causal, not rotated: ascending j.
+__device__ __forceinline__ int contribution_pos(int i, int j, int V, bool causal, bool rotated) {
+    if (causal) return min(i, V - 1) - j;
+    if (!rotated) return j;
+    if (i >= V - 1) return (V - 1) - j;
+    return j <= i ? (i - j) : (i + V - j);
+}
+
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                   const BwdParams p) {
@@ -148,18 +177,23 @@ __global__ void __launch_bounds__(320, 1)
     uint64_t* bar_qfull = bars + 1;
     uint64_t* bar_qempty = bar_qfull + C::QST;
     uint64_t* bar_sfull = bar_qempty + C::QST;
-    uint64_t* bar_pfull = bar_sfull + 1;
-    uint64_t* bar_dqfull = bar_pfull + 1;
+    uint64_t* bar_dpfull = bar_sfull + 1;
+    uint64_t* bar_pfull = bar_dpfull + 1;
+    uint64_t* bar_dsfull = bar_pfull + 1;
+    uint64_t* bar_dqfull = bar_dsfull + 1;
     uint64_t* bar_dqempty = bar_dqfull + 1;
-    uint64_t* bar_dkvfull = bar_dqempty + 1;
+    uint64_t* bar_done = bar_dqempty + 1;
+    uint64_t* bar_go = bar_done + 1;      // [2], alternating by query-block step
+    uint64_t* bar_added = bar_go + 2;     // [2], alternating by query-block step
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SMEM_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::SMEM_MISC + 4);
     int* tile_slot = reinterpret_cast<int*>(smem + C::SMEM_MISC + 8);
-    float* s_lse2 = reinterpret_cast<float*>(smem + C::SMEM_VEC);       // [2][BM]
-    float* s_D = s_lse2 + 2 * C::BM;                                      // [2][BM]
+    volatile int* published = reinterpret_cast<volatile int*>(smem + C::SMEM_MISC + 12);
+    float* s_lse2 = reinterpret_cast<float*>(smem + C::SMEM_VEC);  // [2][BM]
+    float* s_D = s_lse2 + 2 * C::BM;                                 // [2][BM]
 
-    // Tiles are claimed in launch order with an atomic ticket, so a CTA only ever waits (in the
-    // ordered dQ reduction) for tiles that running CTAs claimed earlier: no deadlock.
+    // Tiles are claimed in launch order with an atomic ticket, so a CTA never waits for a tile
+    // that no running CTA has claimed (see contribution_pos for the waits).
     if (threadIdx.x == 0) {
         *tile_slot = atomicAdd(p.tile_counter, 1);
         if (smem_u32(smem) & 1023u) record_error(p.err, kErrInvalidArg);
@@ -167,12 +201,10 @@ __global__ void __launch_bounds__(320, 1)
     __syncthreads();
     const int tile = *tile_slot;
     const int bh = tile / n_kv;
-    // Key block of this tile.  Causal heads run their key blocks from last to first: block j
-    // then reaches query block i after i - j steps, so the order in which blocks arrive at a
-    // query block is j = i, i-1, ..., 0 -- the order the dQ reduction below adds them in.
+    // Causal heads are claimed from their last key block down: block j waits for block j+1.
     const int j = p.causal ? (n_kv - 1 - tile % n_kv) : (tile % n_kv);
     const int b = bh / p.H;
-    const int L = seq_len(p, b, threadIdx.x == 0 && j == 0);
+    const int L = seq_len(p, b, threadIdx.x == 0 && tile % n_kv == 0);
     const int k0 = j * C::BN;
 
     if (k0 >= L) {
@@ -186,9 +218,17 @@ __global__ void __launch_bounds__(320, 1)
         }
         return;
     }
-    const int i_start = p.causal ? j : 0;  // causal: query blocks before the diagonal see none
-    const int n_kv_valid = (L + C::BN - 1) / C::BN;
+    const int V = (L + C::BN - 1) / C::BN;  // key blocks holding at least one visible key
+    // Non-causal heads rotate their query-block order when all V key blocks of a head can be
+    // resident together (the rotated order waits in a cycle j -> j+1 -> ... -> V-1 -> 0).
+    const bool rotated = !p.causal && V <= p.resident_ctas;
+    const int i_start = p.causal ? j : 0;
     const int n_it = n_q - i_start;
+    auto q_block = [&](int it) {
+        if (p.causal) return j + it;
+        if (rotated) { const int i = j + it; return i < n_q ? i : i - n_q; }
+        return it;
+    };
 
     if (threadIdx.x == 0) {
         mbar_init(bar_kv, 1);
@@ -197,11 +237,18 @@ __global__ void __launch_bounds__(320, 1)
             mbar_init(&bar_qempty[s], 1);
         }
         mbar_init(bar_sfull, 1);
-        mbar_init(bar_pfull, C::BN);
+        mbar_init(bar_dpfull, 1);
+        mbar_init(bar_pfull, 256);
+        mbar_init(bar_dsfull, 256);
         mbar_init(bar_dqfull, 1);
-        mbar_init(bar_dqempty, C::BM);
-        mbar_init(bar_dkvfull, 1);
+        mbar_init(bar_dqempty, 128);
+        mbar_init(bar_done, 1);
+        mbar_init(&bar_go[0], 1);
+        mbar_init(&bar_go[1], 1);
+        mbar_init(&bar_added[0], 128);
+        mbar_init(&bar_added[1], 128);
         *abort_flag = 0;
+        *published = 0;
         fence_barrier_init();
     }
     if (warp == 8) {
@@ -218,248 +265,351 @@ __global__ void __launch_bounds__(320, 1)
         *abort_flag = 1;
     };
 
-    if (warp == 9) {
-        // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            prefetch_tensormap(&tmQ);
-            prefetch_tensormap(&tmK);
-            prefetch_tensormap(&tmV);
-            prefetch_tensormap(&tmDO);
-            mbar_arrive_expect_tx(bar_kv, 2 * C::KV_TILE_BYTES);
-            for (int c = 0; c < C::KCH; ++c) {
-                tma_load_3d(smem + C::SMEM_K + c * C::CHUNK_BYTES, &tmK, bar_kv, c * 64, k0, bh);
-                tma_load_3d(smem + C::SMEM_V + c * C::CHUNK_BYTES, &tmV, bar_kv, c * 64, k0, bh);
-            }
-            int it = 0;
-            for (; it < n_it; ++it) {
-                const int s = it % C::QST;
-                const uint32_t ph = (it / C::QST) & 1;
-                const int q0 = (i_start + it) * C::BM;
-                if (!mbar_wait(&bar_qempty[s], ph ^ 1, p.timeout_ns, abort_flag)) { fail(); break; }
-                mbar_arrive_expect_tx(&bar_qfull[s], 2 * C::Q_TILE_BYTES);
-                for (int c = 0; c < C::KCH; ++c) {
-                    tma_load_3d(smem + C::SMEM_Q + s * C::Q_TILE_BYTES + c * C::CHUNK_BYTES, &tmQ,
-                                &bar_qfull[s], c * 64, q0, bh);
-                    tma_load_3d(smem + C::SMEM_DO + s * C::Q_TILE_BYTES + c * C::CHUNK_BYTES,
-                                &tmDO, &bar_qfull[s], c * 64, q0, bh);
-                }
-            }
-            // Do not leave while our copies may still be landing in shared memory.
-            for (int t = max(0, it - C::QST); t < it; ++t)
-                mbar_wait(&bar_qfull[t % C::QST], (t / C::QST) & 1, p.timeout_ns, abort_flag);
-            mbar_wait(bar_kv, 0, p.timeout_ns, abort_flag);
-        }
-    } else if (warp == 8) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idS = idesc_bf16(128, 128, false, false);  // S^T, dP^T
-            constexpr uint32_t idKV = idesc_bf16(128, D, false, true);    // dV, dK (A in TMEM)
-            constexpr uint32_t idQ = idesc_bf16(128, D, true, true);      // dQ = dS K
-            const uint32_t sK = smem_u32(smem + C::SMEM_K);
-            const uint32_t sV = smem_u32(smem + C::SMEM_V);
-            const uint32_t sQ = smem_u32(smem + C::SMEM_Q);
-            const uint32_t sDO = smem_u32(smem + C::SMEM_DO);
-            const uint32_t sDS = smem_u32(smem + C::SMEM_DS);
-            bool ok = mbar_wait(bar_kv, 0, p.timeout_ns, abort_flag);
-            for (int it = 0; ok && it < n_it; ++it) {
-                const int s = it % C::QST;
-                const uint32_t ph = (it / C::QST) & 1;
-                const uint32_t qa = sQ + s * C::Q_TILE_BYTES;
-                const uint32_t da = sDO + s * C::Q_TILE_BYTES;
-                if (!(ok = mbar_wait(&bar_qfull[s], ph, p.timeout_ns, abort_flag))) break;
-                if (it > 0 && !(ok = mbar_wait(bar_dqempty, (it - 1) & 1, p.timeout_ns, abort_flag)))
-                    break;
-                tc_fence_after();
-                // S^T = K Q^T and dP^T = V dO^T: K-major operands, 16-column K steps.
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk / 4) * C::CHUNK_BYTES + (kk % 4) * 32;
-                    mma_ss(tmem + C::TM_A, sdesc_sw128(sK + off, 16, 1024),
-                           sdesc_sw128(qa + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
-                }
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk / 4) * C::CHUNK_BYTES + (kk % 4) * 32;
-                    mma_ss(tmem + C::TM_B, sdesc_sw128(sV + off, 16, 1024),
-                           sdesc_sw128(da + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
-                }
-                tc_commit(bar_sfull);
-                if (!(ok = mbar_wait(bar_pfull, it & 1, p.timeout_ns, abort_flag))) break;
-                tc_fence_after();
-                // dV += P^T dO and dK += dS^T Q: A from tensor memory (16 queries = 8 columns per
-                // K step), B MN-major in shared memory (16 query rows = 2048 bytes per K step).
-#pragma unroll
-                for (int kk = 0; kk < C::BM / 16; ++kk)
-                    mma_ts(tmem + C::TM_DV, tmem + C::TM_A + kk * 8,
-                           sdesc_sw128(da + kk * 2048, C::CHUNK_BYTES, 1024), idKV,
-                           (it > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-                for (int kk = 0; kk < C::BM / 16; ++kk)
-                    mma_ts(tmem + C::TM_DK, tmem + C::TM_B + kk * 8,
-                           sdesc_sw128(qa + kk * 2048, C::CHUNK_BYTES, 1024), idKV,
-                           (it > 0 || kk > 0) ? 1u : 0u);
-                tc_commit(&bar_qempty[s]);
-                // dQ block = dS K: A = dS (queries x keys) read MN-major from the dS^T tile,
-                // B = K MN-major (16 key rows = 2048 bytes per K step).
-#pragma unroll
-                for (int kk = 0; kk < C::BN / 16; ++kk)
-                    mma_ss(tmem + C::TM_A, sdesc_sw128(sDS + kk * 2048, C::CHUNK_BYTES, 1024),
-                           sdesc_sw128(sK + kk * 2048, C::CHUNK_BYTES, 1024), idQ,
-                           kk > 0 ? 1u : 0u);
-                tc_commit(bar_dqfull);
-            }
-            if (!ok) fail();
-            // Always signal the end, then wait for every MMA this thread issued to finish, so
-            // tensor memory is never released under a running MMA (also on the abort path).
-            tc_commit(bar_dkvfull);
-            mbar_wait(bar_dkvfull, 0, p.timeout_ns, abort_flag);
-        }
-    } else if (warp < 4) {
-        // ------------------------------------------------------------ P^T and dS^T
-        const int r = threadIdx.x;  // key row in the block == TMEM lane
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        const int kidx = k0 + r;
-        const bool key_padded = kidx >= L;
-        uint8_t* ds_row = smem + C::SMEM_DS + r * 128;
-        const int sw = r & 7;
-        bool ok = true;
-        for (int it = 0; it < n_it; ++it) {
-            const int i = i_start + it;
-            const int q0 = i * C::BM;
-            const int buf = it & 1;
-            {
-                const int q = q0 + r;
-                s_lse2[buf * C::BM + r] =
-                    q < p.N ? p.lse[(size_t)bh * p.N + q] * kLog2e : INFINITY;
-                s_D[buf * C::BM + r] = q < p.N ? p.Dvec[(size_t)bh * p.N + q] : 0.f;
-            }
-            named_barrier(1, 128);
-            ok = mbar_wait(bar_sfull, it & 1, p.timeout_ns, abort_flag);
-            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-            tc_fence_after();
-            const bool diag = p.causal && (i == j);
-            const float* lse2 = s_lse2 + buf * C::BM;
-            const float* Dv = s_D + buf * C::BM;
-#pragma unroll 1
-            for (int c = 0; c < C::BM / 32; ++c) {
-                uint32_t sv[32], dp[32];
-                tmem_ld32(tmem + lane_base + C::TM_A + c * 32, sv);
-                tmem_ld32(tmem + lane_base + C::TM_B + c * 32, dp);
-                tmem_ld_wait();
-                reg_fence32(sv);
-                reg_fence32(dp);
-                uint32_t pw[16], dw[16];
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const int col = c * 32 + e;
-                    float p0 = ex2(fmaf(__uint_as_float(sv[e]), p.scale_log2, -lse2[col]));
-                    float p1 = ex2(fmaf(__uint_as_float(sv[e + 1]), p.scale_log2, -lse2[col + 1]));
-                    if (key_padded || (diag && r > col)) p0 = 0.f;
-                    if (key_padded || (diag && r > col + 1)) p1 = 0.f;
-                    const float d0 = p0 * (__uint_as_float(dp[e]) - Dv[col]);
-                    const float d1 = p1 * (__uint_as_float(dp[e + 1]) - Dv[col + 1]);
-                    pw[e / 2] = pack_bf16x2(p0, p1);
-                    dw[e / 2] = pack_bf16x2(d0, d1);
-                }
-                // P^T and dS^T as bf16 into tensor memory over the columns already read.
-                tmem_st16(tmem + lane_base + C::TM_A + c * 16, pw);
-                tmem_st16(tmem + lane_base + C::TM_B + c * 16, dw);
-                // dS^T row r into the 128-byte-swizzled shared tile: query chunk c/2, 16-byte
-                // units (c%2)*4 .. +3, unit u stored at position u ^ (r % 8).
-                uint8_t* base = ds_row + (c / 2) * C::CHUNK_BYTES;
-#pragma unroll
-                for (int u4 = 0; u4 < 4; ++u4) {
-                    const int u = (c % 2) * 4 + u4;
-                    *reinterpret_cast<uint4*>(base + ((u ^ sw) << 4)) =
-                        make_uint4(dw[4 * u4], dw[4 * u4 + 1], dw[4 * u4 + 2], dw[4 * u4 + 3]);
-                }
-            }
-            tmem_st_wait();
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(bar_pfull);
-        }
-        if (!ok) fail();
-    } else {
-        // ------------------------------------------------------------ dQ drain, dK/dV epilogue
-        const int r = threadIdx.x - 128;  // query row in the block == TMEM lane
+    if (warp >= 12) {
+        regs_increase<C::REGS_DRAIN>();
+        // ------------------------------------------------------------ dQ drain
+        const int r = threadIdx.x - 384;                // TMEM lane
         const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
         bool ok = true;
         for (int it = 0; it < n_it; ++it) {
-            const int i = i_start + it;
+            const int q0 = q_block(it) * C::BM;
             ok = mbar_wait(bar_dqfull, it & 1, p.timeout_ns, abort_flag);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             tc_fence_after();
-            uint32_t v[D];
+            uint32_t v[128];
+            constexpr int NV = (D == 128) ? 128 : 64;
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) tmem_ld32(tmem + lane_base + C::TM_A + c * 32, v + c * 32);
+            for (int q = 0; q < NV / 32; ++q) tmem_ld32(tmem + lane_base + C::TM_B + 32 * q, v + 32 * q);
             tmem_ld_wait();
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) reg_fence32(v + c * 32);
+            for (int q = 0; q < NV / 32; ++q) reg_fence32(v + 32 * q);
             tc_fence_before();
-            mbar_arrive(bar_dqempty);
-
-            // Ordered reduction into the fp32 accumulator of query block i.  Non-causal: key
-            // blocks add in ascending order (position j).  Causal: descending from the last key
-            // block that sees block i (position jmax - j).  The counter holds the number of
-            // blocks already added; a tile only waits for tiles claimed before it.
-            const int jmax = min(i, n_kv_valid - 1);
-            const int pos = p.causal ? (jmax - j) : j;
-            int* sem = p.sem + (size_t)bh * n_q + i;
-            if (r == 0 && pos > 0) {
-                const uint64_t t0 = globaltimer_ns();
+            mbar_arrive(bar_dqempty);           // B may take the next dP^T
+            ok = mbar_wait(&bar_go[it & 1], (it >> 1) & 1, p.timeout_ns, abort_flag);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            const bool first = contribution_pos(q0 / C::BM, j, V, p.causal != 0, rotated) == 0;
+            float* acc = p.dq_acc + ((size_t)bh * p.N_pad + q0) * D;
+            if constexpr (D == 128) {
+                // dQ^T: lane = feature r, column = query e: a warp covers 32 consecutive
+                // features of one query row, one 128-byte line per instruction.
+                float* dst = acc + r;
+                if (first) {
+#pragma unroll
+                    for (int e = 0; e < 128; ++e) dst[(size_t)e * D] = __uint_as_float(v[e]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 128; ++e) red_add_f32(dst + (size_t)e * D, __uint_as_float(v[e]));
+                }
+            } else {
+                // dQ: lane = query r, 64 features.
+                float* dst = acc + (size_t)r * D;
+                if (first) {
+#pragma unroll
+                    for (int e = 0; e < 64; e += 4)
+                        *reinterpret_cast<float4*>(dst + e) =
+                            make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                                        __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 64; e += 4)
+                        red_add_v4(dst + e, __uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                                   __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+                }
+            }
+            mbar_arrive(&bar_added[it & 1]);    // the ordering thread publishes the count
+        }
+        if (!ok) fail();
+    } else if (warp >= 8) {
+      regs_decrease<C::REGS_OTHER>();
+      if (warp == 9 && lane == 0) {
+        // ------------------------------------------------------------ TMA producer
+        prefetch_tensormap(&tmQ);
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+        prefetch_tensormap(&tmDO);
+        mbar_arrive_expect_tx(bar_kv, 2 * C::KV_TILE_BYTES);
+        for (int c = 0; c < C::KCH; ++c) {
+            tma_load_3d(smem + C::SMEM_K + c * C::CHUNK_BYTES, &tmK, bar_kv, c * 64, k0, bh);
+            tma_load_3d(smem + C::SMEM_V + c * C::CHUNK_BYTES, &tmV, bar_kv, c * 64, k0, bh);
+        }
+        int it = 0;
+        for (; it < n_it; ++it) {
+            const int s = it % C::QST;
+            const uint32_t ph = (it / C::QST) & 1;
+            const int q0 = q_block(it) * C::BM;
+            if (!mbar_wait(&bar_qempty[s], ph ^ 1, p.timeout_ns, abort_flag)) { fail(); break; }
+            mbar_arrive_expect_tx(&bar_qfull[s], 2 * C::Q_TILE_BYTES);
+            for (int c = 0; c < C::KCH; ++c) {
+                tma_load_3d(smem + C::SMEM_Q + s * C::Q_TILE_BYTES + c * C::CHUNK_BYTES, &tmQ,
+                            &bar_qfull[s], c * 64, q0, bh);
+                tma_load_3d(smem + C::SMEM_DO + s * C::Q_TILE_BYTES + c * C::CHUNK_BYTES,
+                            &tmDO, &bar_qfull[s], c * 64, q0, bh);
+            }
+        }
+        // Do not leave while our copies may still be landing in shared memory.
+        for (int t = max(0, it - C::QST); t < it; ++t)
+            mbar_wait(&bar_qfull[t % C::QST], (t / C::QST) & 1, p.timeout_ns, abort_flag);
+        mbar_wait(bar_kv, 0, p.timeout_ns, abort_flag);
+      } else if (warp == 10 && lane == 0) {
+        // ------------------------------------------------------------ dQ add ordering: turns
+        // Step it: wait until key block j is next to add into query block q_block(it) and say
+        // so on bar_go[it & 1].  Publishing is left to warp 11, so this thread never waits for
+        // this CTA's own adds: a turn only ever depends on earlier steps, here and in the
+        // other CTAs (no cycle).  Before step it it waits until warp 11 has passed step it-2,
+        // so no phase of the alternating barrier pairs can be lapped.
+        bool ok = true;
+        for (int it = 0; ok && it < n_it; ++it) {
+            const int i = q_block(it);
+            const int pos = contribution_pos(i, j, V, p.causal != 0, rotated);
+            const int* sem = p.sem + (size_t)bh * n_q + i;
+            const uint64_t t0 = globaltimer_ns();
+            while (it >= 2 && *published < it - 1) {
+                if (*abort_flag || globaltimer_ns() - t0 > p.timeout_ns) { ok = false; break; }
+            }
+            if (!ok) break;
+            if (pos > 0) {
                 while (ld_acquire_gpu(sem) != pos) {
                     if (*abort_flag || globaltimer_ns() - t0 > p.timeout_ns) { ok = false; break; }
                 }
-                if (!ok) fail();
+                if (!ok) break;
             }
-            named_barrier(2, 128);
-            if (*abort_flag) { ok = false; break; }
-            float* dst = p.dq_acc + ((size_t)bh * p.N_pad + (size_t)i * C::BM + r) * D;
-            if (pos == 0) {
-#pragma unroll
-                for (int c = 0; c < D; c += 4)
-                    *reinterpret_cast<float4*>(dst + c) =
-                        make_float4(__uint_as_float(v[c]), __uint_as_float(v[c + 1]),
-                                    __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
-            } else {
-#pragma unroll
-                for (int c = 0; c < D; c += 4)
-                    red_add_v4(dst + c, __uint_as_float(v[c]), __uint_as_float(v[c + 1]),
-                               __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
-            }
-            __threadfence();
-            named_barrier(2, 128);
-            if (r == 0) st_release_gpu(sem, pos + 1);
+            mbar_arrive(&bar_go[it & 1]);
         }
-        if (ok) ok = mbar_wait(bar_dkvfull, 0, p.timeout_ns, abort_flag);
+        if (!ok) fail();
+      } else if (warp == 11 && lane == 0) {
+        // ------------------------------------------------------------ dQ add ordering: counts
+        // Once the drain has issued step it's adds (bar_added), make them visible at GPU scope
+        // and publish the count that lets the next key block add into that query block.
+        bool ok = true;
+        for (int it = 0; it < n_it; ++it) {
+            if (!(ok = mbar_wait(&bar_added[it & 1], (it >> 1) & 1, p.timeout_ns, abort_flag)))
+                break;
+            const int i = q_block(it);
+            fence_acq_rel_gpu();  // the drain's adds, acquired through bar_added
+            st_release_gpu(p.sem + (size_t)bh * n_q + i,
+                           contribution_pos(i, j, V, p.causal != 0, rotated) + 1);
+            *published = it + 1;
+        }
+        if (!ok) fail();
+      } else if (warp == 8 && lane == 0) {
+        // ------------------------------------------------------------ MMA issuer
+        constexpr uint32_t idS = idesc_bf16(128, 128, false, false);  // S^T, dP^T
+        constexpr uint32_t idKV = idesc_bf16(128, D, false, true);    // dV, dK (A in TMEM)
+        constexpr uint32_t idQ = idesc_bf16(128, D == 128 ? 128 : 64, true, true);  // dQ^T / dQ
+        const uint32_t sK = smem_u32(smem + C::SMEM_K);
+        const uint32_t sV = smem_u32(smem + C::SMEM_V);
+        const uint32_t sQ = smem_u32(smem + C::SMEM_Q);
+        const uint32_t sDO = smem_u32(smem + C::SMEM_DO);
+        const uint32_t sDS = smem_u32(smem + C::SMEM_DS);
+        bool ok = mbar_wait(bar_kv, 0, p.timeout_ns, abort_flag);
+        for (int it = 0; ok && it < n_it; ++it) {
+            const int s = it % C::QST;
+            const uint32_t ph = (it / C::QST) & 1;
+            const uint32_t qa = sQ + s * C::Q_TILE_BYTES;
+            const uint32_t da = sDO + s * C::Q_TILE_BYTES;
+            if (!(ok = mbar_wait(&bar_qfull[s], ph, p.timeout_ns, abort_flag))) break;
+            tc_fence_after();
+            // S^T = K Q^T: K-major operands, 16-column K steps (32 bytes inside a swizzled row,
+            // then the next 64-column chunk).
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk / 4) * C::CHUNK_BYTES + (kk % 4) * 32;
+                mma_ss(tmem + C::TM_A, sdesc_sw128(sK + off, 16, 1024),
+                       sdesc_sw128(qa + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(bar_sfull);
+            // dP^T = V dO^T into B, once the previous dQ block has been drained from B.
+            if (it > 0 && !(ok = mbar_wait(bar_dqempty, (it - 1) & 1, p.timeout_ns, abort_flag)))
+                break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk / 4) * C::CHUNK_BYTES + (kk % 4) * 32;
+                mma_ss(tmem + C::TM_B, sdesc_sw128(sV + off, 16, 1024),
+                       sdesc_sw128(da + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(bar_dpfull);
+            // dV += P^T dO: A = P^T in tensor memory (16 queries = 8 columns per K step),
+            // B = dO MN-major (16 query rows = 2048 bytes per K step).
+            if (!(ok = mbar_wait(bar_pfull, it & 1, p.timeout_ns, abort_flag))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < C::BM / 16; ++kk)
+                mma_ts(tmem + C::TM_DV, tmem + C::TM_A + kk * 8,
+                       sdesc_sw128(da + kk * 2048, C::CHUNK_BYTES, 1024), idKV,
+                       (it > 0 || kk > 0) ? 1u : 0u);
+            // dK += dS^T Q, same shapes.
+            if (!(ok = mbar_wait(bar_dsfull, it & 1, p.timeout_ns, abort_flag))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < C::BM / 16; ++kk)
+                mma_ts(tmem + C::TM_DK, tmem + C::TM_B + kk * 8,
+                       sdesc_sw128(qa + kk * 2048, C::CHUNK_BYTES, 1024), idKV,
+                       (it > 0 || kk > 0) ? 1u : 0u);
+            tc_commit(&bar_qempty[s]);
+            // The dQ block into B; K steps of 16 keys = 2048 bytes of both tiles, both
+            // operands MN-major.
+            if constexpr (D == 128) {
+                // dQ^T = K^T dS^T: A = K^T (M = feature), B = dS^T (N = query).
+#pragma unroll
+                for (int kk = 0; kk < C::BN / 16; ++kk)
+                    mma_ss(tmem + C::TM_B, sdesc_sw128(sK + kk * 2048, C::CHUNK_BYTES, 1024),
+                           sdesc_sw128(sDS + kk * 2048, C::CHUNK_BYTES, 1024), idQ,
+                           kk > 0 ? 1u : 0u);
+            } else {
+                // dQ = dS K: A = dS (M = query, from the dS^T tile), B = K (N = feature).
+#pragma unroll
+                for (int kk = 0; kk < C::BN / 16; ++kk)
+                    mma_ss(tmem + C::TM_B, sdesc_sw128(sDS + kk * 2048, C::CHUNK_BYTES, 1024),
+                           sdesc_sw128(sK + kk * 2048, C::CHUNK_BYTES, 1024), idQ,
+                           kk > 0 ? 1u : 0u);
+            }
+            tc_commit(bar_dqfull);
+        }
+        if (!ok) fail();
+        // Wait for every MMA issued here before tensor memory can be released.
+        tc_commit(bar_done);
+        mbar_wait(bar_done, 0, p.timeout_ns, abort_flag);
+      }
+    } else {
+        regs_increase<C::REGS_COMPUTE>();
+        // ------------------------------------------------------------ compute warpgroups
+        const int h = warp / 4;                          // query-column half
+        const int r = threadIdx.x % 128;                 // TMEM lane
+        const int ct = threadIdx.x;                      // 0..255
+        const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
+        const int kidx = k0 + r;
+        const bool key_padded = kidx >= L;
+        uint8_t* ds_row = smem + C::SMEM_DS + h * C::CHUNK_BYTES + r * 128;
+        const int sw = r & 7;
+        const float c = p.scale_log2;
+
+        // lse * log2(e) and D of query block q_block(it) into buffer it & 1 (threads 0..127 the
+        // lse values, 128..255 the D values); +inf / 0 past N so those queries get P = 0.
+        // The global load is issued one iteration ahead (load_vectors) and stored to shared
+        // memory at the end of the iteration (store_vectors), so its latency stays hidden.
+        float staged = 0.f;
+        auto load_vectors = [&](int it) {
+            const int q = q_block(it) * C::BM + (ct & 127);
+            if (ct < 128) staged = q < p.N ? p.lse[(size_t)bh * p.N + q] * kLog2e : INFINITY;
+            else staged = q < p.N ? p.Dvec[(size_t)bh * p.N + q] : 0.f;
+        };
+        auto store_vectors = [&](int it) {
+            if (ct < 128) s_lse2[(it & 1) * C::BM + ct] = staged;
+            else s_D[(it & 1) * C::BM + (ct - 128)] = staged;
+        };
+        load_vectors(0);
+        store_vectors(0);
+        named_barrier(1, 256);
+
+        bool ok = true;
+        for (int it = 0; it < n_it; ++it) {
+            const int i = q_block(it);
+            const int q0 = i * C::BM;
+            const float* lse2 = s_lse2 + (it & 1) * C::BM + 64 * h;
+            const float* Dv = s_D + (it & 1) * C::BM + 64 * h;
+            if (it + 1 < n_it) load_vectors(it + 1);  // stored at the end of this iteration
+            const bool diag = p.causal && (i == j);
+
+            // ---------------- P phase
+            ok = mbar_wait(bar_sfull, it & 1, p.timeout_ns, abort_flag);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+            float P[64];
+            {
+                uint32_t sv[64];
+                tmem_ld32(tmem + lane_base + C::TM_A + 64 * h, sv);
+                tmem_ld32(tmem + lane_base + C::TM_A + 64 * h + 32, sv + 32);
+                tmem_ld_wait();
+                reg_fence32(sv);
+                reg_fence32(sv + 32);
+#pragma unroll
+                for (int e = 0; e < 64; e += 2) {
+                    const float2 x = ffma2(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])),
+                                           make_float2(c, c), make_float2(-lse2[e], -lse2[e + 1]));
+                    P[e] = ex2(x.x);
+                    P[e + 1] = ex2(x.y);
+                }
+                if (key_padded || diag) {
+#pragma unroll
+                    for (int e = 0; e < 64; ++e)
+                        if (key_padded || r > 64 * h + e) P[e] = 0.f;
+                }
+            }
+            named_barrier(1, 256);  // every S^T column read before P^T overwrites columns
+            {
+                uint32_t pw[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) pw[e] = pack_bf16x2(P[2 * e], P[2 * e + 1]);
+                tmem_st32(tmem + lane_base + C::TM_A + 32 * h, pw);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(bar_pfull);
+
+            // ---------------- dS phase
+            ok = mbar_wait(bar_dpfull, it & 1, p.timeout_ns, abort_flag);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t dw[32];
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t dp[32];
+                tmem_ld32(tmem + lane_base + C::TM_B + 64 * h + 32 * half, dp);
+                tmem_ld_wait();
+                reg_fence32(dp);
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    const int ee = 32 * half + e;
+                    const float d0 = P[ee] * (__uint_as_float(dp[e]) - Dv[ee]);
+                    const float d1 = P[ee + 1] * (__uint_as_float(dp[e + 1]) - Dv[ee + 1]);
+                    dw[ee / 2] = pack_bf16x2(d0, d1);
+                }
+            }
+            // Next block's lse / D into the other buffer: every thread has passed this
+            // iteration's first barrier, so nobody still reads that buffer, and the barrier
+            // below orders these stores before the next iteration's reads.
+            if (it + 1 < n_it) store_vectors(it + 1);
+            named_barrier(1, 256);  // every dP^T column read before dS^T overwrites columns
+            tmem_st32(tmem + lane_base + C::TM_B + 32 * h, dw);
+            // dS^T row r, queries [64h, 64h+64) = one 128-byte row of query chunk h; 16-byte
+            // unit u sits at position u ^ (r % 8) (the 128-byte swizzle the MMA reads).
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                *reinterpret_cast<uint4*>(ds_row + ((u ^ sw) << 4)) =
+                    make_uint4(dw[4 * u], dw[4 * u + 1], dw[4 * u + 2], dw[4 * u + 3]);
+            tmem_st_wait();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar_dsfull);
+
+        }
+
+        // ---------------- epilogue: dV (warpgroup 0) and dK * scale (warpgroup 1)
+        if (ok) ok = mbar_wait(bar_done, 0, p.timeout_ns, abort_flag);  // every MMA finished
         if (__all_sync(0xffffffffu, ok)) {
             tc_fence_after();
-            const int kidx = k0 + r;
             const bool in_range = kidx < p.N;
             const size_t off = ((size_t)bh * p.N + (in_range ? kidx : 0)) * D;
+            const uint32_t col0 = h ? C::TM_DK : C::TM_DV;
+            const float mul = h ? p.scale : 1.0f;
+            __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(h ? p.dk : p.dv) + off;
 #pragma unroll
-            for (int which = 0; which < 2; ++which) {
-                const uint32_t col0 = which ? C::TM_DK : C::TM_DV;
-                const float mul = which ? p.scale : 1.0f;
-                __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(which ? p.dk : p.dv) + off;
+            for (int q = 0; q < D / 32; ++q) {
+                uint32_t x[32];
+                tmem_ld32(tmem + lane_base + col0 + q * 32, x);
+                tmem_ld_wait();
+                reg_fence32(x);
+                uint32_t w[16];
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t x[32];
-                    tmem_ld32(tmem + lane_base + col0 + c * 32, x);
-                    tmem_ld_wait();
-                    reg_fence32(x);
-                    uint32_t w[16];
+                for (int e = 0; e < 16; ++e)
+                    w[e] = pack_bf16x2(__uint_as_float(x[2 * e]) * mul,
+                                       __uint_as_float(x[2 * e + 1]) * mul);
+                if (in_range) {
+                    uint4* dst = reinterpret_cast<uint4*>(out + q * 32);
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        w[e] = pack_bf16x2(__uint_as_float(x[2 * e]) * mul,
-                                           __uint_as_float(x[2 * e + 1]) * mul);
-                    if (in_range) {
-                        uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
-                    }
+                    for (int e = 0; e < 4; ++e)
+                        dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
                 }
             }
         } else {

@@ -41,6 +41,7 @@ struct BwdParams {
     float scale;
     float scale_log2;
     int causal;
+    int resident_ctas;     // CTAs of the main kernel that can be resident at once (1 per SM)
     uint64_t timeout_ns;
 };
 

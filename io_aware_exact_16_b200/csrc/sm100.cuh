@@ -281,6 +281,19 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
                  "f"(d)
                  : "memory");
 }
+// fp32 add of one float into global memory (no return value).
+__device__ __forceinline__ void red_add_f32(float* p, float a) {
+    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(a) : "memory");
+}
+// Orders this thread's (and, through a preceding barrier, its CTA's) prior memory accesses
+// before its later ones at GPU scope.
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+// Arrives on named barrier `id` (expecting `count` threads) without waiting.
+__device__ __forceinline__ void named_barrier_arrive(int id, int count) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 // Named barrier over `count` threads (a multiple of 32) of this CTA.
 __device__ __forceinline__ void named_barrier(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
