@@ -81,10 +81,10 @@ FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, fl
 
 /*
  * Bytes of device workspace fa_bwd needs for these sizes (0 if the sizes are invalid).
- * The workspace holds D = rowsum(dO * O) (fp32 [B, H, N]), the fp32 dQ accumulator
- * ([B, H, N_pad, d] with N_pad = N rounded up to 128), the per-(b, h, query-block) ordering
- * counters of the deterministic dQ reduction and a tile counter.  Its contents need not be
- * initialised; fa_bwd clears what it uses.
+ * The workspace holds D = rowsum(dO * O) and |dO_i| (fp32 [B, H, N] each), per-128-row-chunk
+ * maxima of |v_j| and |k_jl| (fp32 [B, H, N_pad / 128, 2]) and the int32 fixed-point dQ
+ * accumulator ([B, H, N_pad, d]), N_pad = N rounded up to 128.  Its contents need not be
+ * initialised; fa_bwd writes everything it reads.
  */
 FA_API size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 
@@ -98,8 +98,10 @@ FA_API size_t fa_bwd_workspace_size(int B, int H, int N, int d);
  *   dq, dk, dv     out: bf16 [B, H, N, d], fully overwritten
  *   workspace      scratch of at least fa_bwd_workspace_size(B, H, N, d) bytes, 16-byte
  *                  aligned, owned by the caller, not used concurrently by another call.
- * The dQ sum over key blocks runs in a fixed order, so repeated calls on the same inputs
- * give bitwise identical dq, dk, dv.
+ * The dQ sum over key blocks is exact integer (fixed-point) arithmetic: each key block's
+ * contribution to query row i is rounded once to 2^-30 of an a-priori bound of row i
+ * (2 |dO_i| max_j |v_j| max |k|) and the integer sum does not depend on the order in which
+ * key blocks arrive, so repeated calls on the same inputs give bitwise identical dq, dk, dv.
  */
 FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
                  const float* lse, void* dq, void* dk, void* dv,

@@ -108,18 +108,6 @@ bool make_bf16_map(CUtensorMap* map, const void* base, int d, int N, int BH, int
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool make_f32_map(CUtensorMap* map, const void* base, int d, int N_pad, int BH, int box_rows) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return false;
-    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N_pad, (cuuint64_t)BH};
-    cuuint64_t strides[2] = {(cuuint64_t)d * 4, (cuuint64_t)N_pad * d * 4};
-    cuuint32_t box[3] = {32, (cuuint32_t)box_rows, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides,
-               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace fa
 
 using namespace fa;
@@ -179,10 +167,10 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
     const size_t Np = (size_t)pad128(N);
     size_t bytes = 0;
     auto add = [&](size_t n) { bytes += (n + 255) / 256 * 256; };
-    add(BH * N * sizeof(float));           // D
-    add(BH * Np * d * sizeof(float));      // dQ accumulator
-    add(BH * (Np / 128) * sizeof(int));    // ordering counters
-    add(sizeof(int));                      // tile counter
+    add(BH * N * sizeof(float));             // D
+    add(BH * N * sizeof(float));             // |dO_i|
+    add(BH * (Np / 128) * 2 * sizeof(float)); // per-chunk maxima of |v_j| and |k_jl|
+    add(BH * Np * d * sizeof(int));          // fixed-point dQ accumulator
     return bytes;
 }
 
@@ -215,13 +203,15 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
     p.o = o;
     p.dO = dO;
     p.lse = lse;
+    p.k = k;
+    p.v = v;
     p.dq = dq;
     p.dk = dk;
     p.dv = dv;
     p.Dvec = static_cast<float*>(take((size_t)BH * N * sizeof(float)));
-    p.dq_acc = static_cast<float*>(take((size_t)BH * Np * d * sizeof(float)));
-    p.sem = static_cast<int*>(take((size_t)BH * (Np / 128) * sizeof(int)));
-    p.tile_counter = static_cast<int*>(take(sizeof(int)));
+    p.dOnorm = static_cast<float*>(take((size_t)BH * N * sizeof(float)));
+    p.headmax = static_cast<float*>(take((size_t)BH * (Np / 128) * 2 * sizeof(float)));
+    p.dq_acc = static_cast<int*>(take((size_t)BH * Np * d * sizeof(int)));
     p.seqlens = seqlens;
     p.err = dev->err_flag;
     p.B = B;
@@ -231,16 +221,13 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
     p.scale = scale;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
-    p.resident_ctas = dev->num_sms;
     p.timeout_ns = g_timeout_ns.load();
 
-    CUtensorMap tq, tk, tv, tdo, tacc;
+    CUtensorMap tq, tk, tv, tdo;
     if (!make_bf16_map(&tq, q, d, N, BH, 128) || !make_bf16_map(&tk, k, d, N, BH, 128) ||
-        !make_bf16_map(&tv, v, d, N, BH, 128) || !make_bf16_map(&tdo, dO, d, N, BH, 128) ||
-        !make_f32_map(&tacc, p.dq_acc, d, Np, BH, 128))
+        !make_bf16_map(&tv, v, d, N, BH, 128) || !make_bf16_map(&tdo, dO, d, N, BH, 128))
         return FA_ERR_CUDA;
-    if (launch_bwd(d, tq, tk, tv, tdo, tacc, p, dev->num_sms,
-                   reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    if (launch_bwd(d, tq, tk, tv, tdo, p, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
         return FA_ERR_CUDA;
     return FA_OK;
 }

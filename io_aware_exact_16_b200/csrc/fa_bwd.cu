@@ -9,12 +9,23 @@
 //   dK = scale dS^T Q                 dQ = scale dS K
 //
 // Three kernels run in order on one stream:
-//   fa_bwd_pre_kernel   D = rowsum(dO * O) in fp32; clears the ordering counters
+//   fa_bwd_pre_kernel   per row D = rowsum(dO * O) and |dO_i|; per 128-row chunk the largest
+//                       |v_j| and |k_jl|; clears the dQ accumulator
 //   fa_bwd_kernel       one CTA per 128-key block: recomputes S^T, P^T, dP^T, dS^T per
 //                       128-query block with tcgen05 MMAs, accumulates dK, dV in tensor memory
-//                       and adds its dQ block contribution into an fp32 accumulator in a fixed
-//                       key-block order (deterministic)
+//                       and adds its dQ contribution into the accumulator
 //   fa_bwd_dq_kernel    dQ = scale * accumulator -> bf16
+//
+// Deterministic dQ.  Every key block adds a contribution dS_ib K_b to every query row i it
+// sees.  Those contributions are added in integer fixed point, so the sum does not depend on
+// the order in which key blocks arrive and repeated runs are bitwise identical, with no
+// ordering between CTAs.  Row i uses the scale s_i = 2^floor(log2(2^30 / bound_i)), where
+//     bound_i = 2 |dO_i| max_j |v_j| max_{j,l} |k_jl|
+// bounds every partial sum: sum_j |dS_ij| = sum_j P_ij |dP_ij - D_i| <= 2 |dO_i| max_j |v_j|
+// (|dP_ij| <= |dO_i||v_j|, |D_i| <= |dO_i||O_i| and O_i is a convex combination of the v_j), and
+// each feature of sum_j dS_ij k_j is at most that times max |k_jl|.  Sums therefore stay below
+// 2^30 (+ one rounding per key block) and never overflow int32; each contribution is rounded
+// once, to 2^-30 bound_i.
 //
 // Main-kernel warp roles (512 threads = 4 warpgroups):
 //   warps 0-7   compute: warpgroup h owns query columns [64h, 64h+64) of every block; thread
@@ -25,22 +36,20 @@
 //               dV (warpgroup 0) and dK (warpgroup 1).
 //   warp  8     MMA issue (one thread) + TMEM allocation
 //   warp  9     TMA producer (one thread)
-//   warp  10    ordering of the dQ adds, turns (one thread): waits until it is this key block's
-//               turn to add into query block i and says so (bar_go)
-//   warp  11    ordering of the dQ adds, counts (one thread): once the adds are issued
-//               (bar_added), fences and publishes the new count; a separate thread so that
-//               neither the fence nor this CTA's own adds ever hold up a turn
-//   warps 12-15 dQ drain: copy the dQ block out of tensor memory, free it, add it to the
-//               fp32 accumulator.  For d = 128 the block is held transposed (dQ^T = K^T dS^T,
-//               lane = feature, column = query), so each warp adds whole 128-byte lines; for
-//               d = 64 it is dQ = dS K (lane = query) added with 16-byte vector adds.
+//   warps 10-11 idle
+//   warps 12-15 dQ drain: copy the dQ block out of tensor memory, free it, convert it to fixed
+//               point and add it to the accumulator with integer atomics.  For d = 128 the
+//               block is held transposed (dQ^T = K^T dS^T: lane = feature, column = query) so
+//               each warp instruction adds one 128-byte line; for d = 64 it is dQ = dS K (lane =
+//               query) and goes through a per-warp shared-memory transpose to the same pattern.
 // Registers: warpgroup 2 gives its share to warpgroups 0, 1 and 3 (setmaxnreg).
 // Tensor memory (512 columns):
 //   A [0,128)   S^T (fp32) -> P^T (bf16, columns [0,64))
 //   B [128,256) dP^T (fp32) -> dS^T (bf16, [128,192)) -> the dQ block (fp32)
 //   dV [256, 256+d)   dK [256+d, 256+2d)
 // Shared memory: K_j, V_j (once), a 2-stage ring of Q_i / dO_i, dS^T (bf16, 128-byte
-// swizzled, an operand of the dQ MMA), lse*log2(e) and D of the query blocks.
+// swizzled, an operand of the dQ MMA), lse*log2(e), D and the fixed-point scales of the query
+// blocks (and for d = 64 the drain's transpose buffers).
 #include "fa_internal.h"
 #include "sm100.cuh"
 
@@ -66,13 +75,16 @@ struct BwdCfg {
     static constexpr int SMEM_Q = SMEM_V + KV_TILE_BYTES;
     static constexpr int SMEM_DO = SMEM_Q + QST * Q_TILE_BYTES;
     static constexpr int SMEM_DS = SMEM_DO + QST * Q_TILE_BYTES;
-    static constexpr int SMEM_VEC = SMEM_DS + DS_BYTES;       // [2][128] lse2, [2][128] D
-    static constexpr int SMEM_BAR = SMEM_VEC + 4 * BM * 4;
-    static constexpr int NUM_BARS = 1 + 2 * QST + 11;
+    static constexpr int SMEM_VEC = SMEM_DS + DS_BYTES;        // [2][128] lse2, [2][128] D
+    static constexpr int SMEM_SCALE = SMEM_VEC + 4 * BM * 4;   // [128] fixed-point scales
+    static constexpr int SMEM_XPOSE = SMEM_SCALE + BM * 4;     // d = 64: 4 x [32][33] int32
+    static constexpr int XPOSE_BYTES = (D == 64) ? 4 * 32 * 33 * 4 : 0;
+    static constexpr int SMEM_BAR = SMEM_XPOSE + XPOSE_BYTES;
+    static constexpr int NUM_BARS = 1 + 2 * QST + 7;
     static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
-    static constexpr int SMEM_BYTES = SMEM_MISC + 16;  // tmem address, abort, tile, progress
+    static constexpr int SMEM_BYTES = SMEM_MISC + 16;  // tmem address, abort flag
     static constexpr int THREADS = 512;
-    // 2 x 160 (compute) + 56 (MMA / TMA / ordering) + 136 (drain) = 4 x 128 launched
+    // 2 x 160 (compute) + 56 (MMA / TMA) + 136 (drain) = 4 x 128 launched
     static constexpr uint32_t REGS_COMPUTE = 160, REGS_OTHER = 56, REGS_DRAIN = 136;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t TM_A = 0, TM_B = 128, TM_DV = 256, TM_DK = 256 + D;
@@ -94,71 +106,139 @@ __device__ __forceinline__ int seq_len(const BwdParams& p, int b, bool report) {
     return L;
 }
 
+// Head constant 2 max_j |v_j| max_{j,l} |k_jl| from the per-chunk maxima (same arithmetic in
+// every kernel that needs it, so every kernel derives the same scales).
+__device__ __forceinline__ float head_bound_factor(const BwdParams& p, int bh) {
+    const int chunks = p.N_pad / 128;
+    const float* hm = p.headmax + (size_t)bh * chunks * 2;
+    float vmax = 0.f, kmax = 0.f;
+    for (int c = 0; c < chunks; ++c) {
+        vmax = fmaxf(vmax, hm[2 * c]);
+        kmax = fmaxf(kmax, hm[2 * c + 1]);
+    }
+    return 2.0f * vmax * kmax;
+}
+
+// Fixed-point scale of a query row: the largest power of two s with s * bound <= 2^30;
+// 0 when the bound is 0 (then every contribution of the row is 0).
+__device__ __forceinline__ float fixed_point_scale(float dO_norm, float head_factor) {
+    const float bound = dO_norm * head_factor;
+    if (!(bound > 0.f)) return 0.f;
+    const float x = 1073741824.0f / bound;
+    if (!(x <= 3.0e38f)) return 0.f;
+    return __int_as_float(__float_as_int(x) & 0x7F800000);  // 2^floor(log2 x), exact
+}
+
 // ---------------------------------------------------------------------------- preprocess
-// D[row] = sum_k dO[row, k] * O[row, k] in fp32.  16 threads per row for d = 128 (8 for d = 64),
-// each reading 16 bytes of dO and O.  Also clears the ordering counters and the tile counter.
+// Grid (N_pad / 128 chunks, B*H).  Per row: D = dO . O (fp32) and |dO|; per chunk: the largest
+// |v_j| and |k_jl| of its visible key rows (j < L_b); and the chunk's rows of the dQ
+// accumulator set to zero.  TPR threads per row, each reading 16 bytes of every tensor.
 template <int D>
-__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p, int rows, int n_sem) {
-    constexpr int TPR = D / 8;  // threads per row
-    const int gtid = blockIdx.x * blockDim.x + threadIdx.x;
-    const int row = gtid / TPR;
-    const int part = gtid % TPR;
-    float acc = 0.f;
-    if (row < rows) {
-        const uint4 a = reinterpret_cast<const uint4*>(p.dO)[(size_t)row * TPR + part];
-        const uint4 o = reinterpret_cast<const uint4*>(p.o)[(size_t)row * TPR + part];
-        const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
-        const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&o);
+__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p) {
+    constexpr int TPR = D / 8;               // threads per row
+    constexpr int RPP = 256 / TPR;           // rows per pass
+    const int chunk = blockIdx.x;
+    const int bh = blockIdx.y;
+    const int part = threadIdx.x % TPR;
+    // Only keys some query can see enter the bound (padded keys contribute nothing to dQ).
+    const int L = seq_len(p, bh / p.H, false);
+    float vmax = 0.f, kmax = 0.f;
+    for (int rr = threadIdx.x / TPR; rr < 128; rr += RPP) {
+        const int n = chunk * 128 + rr;
+        float dd = 0.f, nn = 0.f, vv = 0.f, ka = 0.f;
+        if (n < p.N) {
+            const size_t off = ((size_t)bh * p.N + n) * TPR + part;
+            const uint4 a = reinterpret_cast<const uint4*>(p.dO)[off];
+            const uint4 o = reinterpret_cast<const uint4*>(p.o)[off];
+            const uint4 v = reinterpret_cast<const uint4*>(p.v)[off];
+            const uint4 k = reinterpret_cast<const uint4*>(p.k)[off];
+            const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+            const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&o);
+            const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+            const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&k);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 fa = __bfloat1622float2(a2[i]);
-            const float2 fo = __bfloat1622float2(o2[i]);
-            acc = fmaf(fa.x, fo.x, acc);
-            acc = fmaf(fa.y, fo.y, acc);
+            for (int i = 0; i < 4; ++i) {
+                const float2 fa = __bfloat1622float2(a2[i]);
+                const float2 fo = __bfloat1622float2(o2[i]);
+                const float2 fv = __bfloat1622float2(v2[i]);
+                const float2 fk = __bfloat1622float2(k2[i]);
+                dd = fmaf(fa.x, fo.x, fmaf(fa.y, fo.y, dd));
+                nn = fmaf(fa.x, fa.x, fmaf(fa.y, fa.y, nn));
+                vv = fmaf(fv.x, fv.x, fmaf(fv.y, fv.y, vv));
+                ka = fmaxf(ka, fmaxf(fabsf(fk.x), fabsf(fk.y)));
+            }
+        }
+#pragma unroll
+        for (int off = TPR / 2; off > 0; off >>= 1) {
+            dd += __shfl_xor_sync(0xffffffffu, dd, off);
+            nn += __shfl_xor_sync(0xffffffffu, nn, off);
+            vv += __shfl_xor_sync(0xffffffffu, vv, off);
+            ka = fmaxf(ka, __shfl_xor_sync(0xffffffffu, ka, off));
+        }
+        if (n < p.N && part == 0) {
+            p.Dvec[(size_t)bh * p.N + n] = dd;
+            p.dOnorm[(size_t)bh * p.N + n] = sqrtf(nn);
+        }
+        if (n < L) {
+            vmax = fmaxf(vmax, sqrtf(vv));
+            kmax = fmaxf(kmax, ka);
         }
     }
 #pragma unroll
-    for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (row < rows && part == 0) p.Dvec[row] = acc;
-    for (int i = gtid; i < n_sem; i += gridDim.x * blockDim.x) p.sem[i] = 0;
-    if (gtid == 0) *p.tile_counter = 0;
+    for (int off = 16; off > 0; off >>= 1) {
+        vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
+        kmax = fmaxf(kmax, __shfl_xor_sync(0xffffffffu, kmax, off));
+    }
+    __shared__ float red[2][8];
+    if (threadIdx.x % 32 == 0) {
+        red[0][threadIdx.x / 32] = vmax;
+        red[1][threadIdx.x / 32] = kmax;
+    }
+    // zero this chunk's 128 rows of the accumulator
+    int4* acc = reinterpret_cast<int4*>(p.dq_acc + ((size_t)bh * p.N_pad + (size_t)chunk * 128) * D);
+    for (int i = threadIdx.x; i < 128 * D / 4; i += 256) acc[i] = make_int4(0, 0, 0, 0);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float a = 0.f, b = 0.f;
+        for (int w = 0; w < 8; ++w) {
+            a = fmaxf(a, red[0][w]);
+            b = fmaxf(b, red[1][w]);
+        }
+        float* hm = p.headmax + ((size_t)bh * (p.N_pad / 128) + chunk) * 2;
+        hm[0] = a;
+        hm[1] = b;
+    }
 }
 
 // ---------------------------------------------------------------------------- dQ convert
-// dq = bf16(scale * dq_acc) for the N real rows of every head; 8 elements per thread.
+// Grid (N_pad / 128 chunks, B*H): dq = bf16(scale * acc / s_i) for the chunk's real rows.
 template <int D>
-__global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const BwdParams p, long long total8) {
-    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= total8) return;
-    const long long e = i * 8;               // element index in [BH, N, D]
-    const long long row = e / D;             // bh * N + n
-    const int col = (int)(e % D);
-    const long long bh = row / p.N;
-    const long long n = row % p.N;
-    const float4* src =
-        reinterpret_cast<const float4*>(p.dq_acc + ((bh * p.N_pad + n) * D + col));
-    const float4 x = src[0], y = src[1];
-    uint4 out;
-    out.x = pack_bf16x2(x.x * p.scale, x.y * p.scale);
-    out.y = pack_bf16x2(x.z * p.scale, x.w * p.scale);
-    out.z = pack_bf16x2(y.x * p.scale, y.y * p.scale);
-    out.w = pack_bf16x2(y.z * p.scale, y.w * p.scale);
-    reinterpret_cast<uint4*>(p.dq)[i] = out;
+__global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const BwdParams p) {
+    const int chunk = blockIdx.x;
+    const int bh = blockIdx.y;
+    __shared__ float s_factor;
+    if (threadIdx.x == 0) s_factor = head_bound_factor(p, bh);
+    __syncthreads();
+    const float factor = s_factor;
+    constexpr int PER_ROW = D / 8;  // 8 elements per thread-step
+    for (int i = threadIdx.x; i < 128 * PER_ROW; i += 256) {
+        const int rr = i / PER_ROW, c8 = (i % PER_ROW) * 8;
+        const int n = chunk * 128 + rr;
+        if (n >= p.N) continue;
+        const float s = fixed_point_scale(p.dOnorm[(size_t)bh * p.N + n], factor);
+        const float mul = s > 0.f ? p.scale / s : 0.f;  // 1 / s is a power of two: exact
+        const int4* src = reinterpret_cast<const int4*>(p.dq_acc + ((size_t)bh * p.N_pad + n) * D + c8);
+        const int4 x = src[0], y = src[1];
+        uint4 out;
+        out.x = pack_bf16x2((float)x.x * mul, (float)x.y * mul);
+        out.y = pack_bf16x2((float)x.z * mul, (float)x.w * mul);
+        out.z = pack_bf16x2((float)y.x * mul, (float)y.y * mul);
+        out.w = pack_bf16x2((float)y.z * mul, (float)y.w * mul);
+        *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.dq) + ((size_t)bh * p.N + n) * D + c8) = out;
+    }
 }
 
 // ---------------------------------------------------------------------------- main kernel
-// Position of key block j in the fixed order in which key blocks add into query block i.
-// Causal: blocks visit i from j upwards, so they reach i in the order j = jmax, jmax-1, ..., 0.
-// Non-causal, rotated: block j visits i = j, j+1, ..., n-1, 0, ..., j-1 and reaches i at step
-// (i - j) mod n, so the order is j = i, i-1, ..., 0, V-1, ..., i+1 (V = key blocks present).
-// Non-causal, not rotated: ascending j.
-__device__ __forceinline__ int contribution_pos(int i, int j, int V, bool causal, bool rotated) {
-    if (causal) return min(i, V - 1) - j;
-    if (!rotated) return j;
-    if (i >= V - 1) return (V - 1) - j;
-    return j <= i ? (i - j) : (i + V - j);
-}
-
 template <int D>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -183,28 +263,18 @@ __global__ void __launch_bounds__(512, 1)
     uint64_t* bar_dqfull = bar_dsfull + 1;
     uint64_t* bar_dqempty = bar_dqfull + 1;
     uint64_t* bar_done = bar_dqempty + 1;
-    uint64_t* bar_go = bar_done + 1;      // [2], alternating by query-block step
-    uint64_t* bar_added = bar_go + 2;     // [2], alternating by query-block step
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SMEM_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::SMEM_MISC + 4);
-    int* tile_slot = reinterpret_cast<int*>(smem + C::SMEM_MISC + 8);
-    volatile int* published = reinterpret_cast<volatile int*>(smem + C::SMEM_MISC + 12);
-    float* s_lse2 = reinterpret_cast<float*>(smem + C::SMEM_VEC);  // [2][BM]
-    float* s_D = s_lse2 + 2 * C::BM;                                 // [2][BM]
+    float* s_lse2 = reinterpret_cast<float*>(smem + C::SMEM_VEC);    // [2][BM]
+    float* s_D = s_lse2 + 2 * C::BM;                                   // [2][BM]
+    float* s_scale = reinterpret_cast<float*>(smem + C::SMEM_SCALE);  // [BM]
 
-    // Tiles are claimed in launch order with an atomic ticket, so a CTA never waits for a tile
-    // that no running CTA has claimed (see contribution_pos for the waits).
-    if (threadIdx.x == 0) {
-        *tile_slot = atomicAdd(p.tile_counter, 1);
-        if (smem_u32(smem) & 1023u) record_error(p.err, kErrInvalidArg);
-    }
-    __syncthreads();
-    const int tile = *tile_slot;
+    if (threadIdx.x == 0 && (smem_u32(smem) & 1023u)) record_error(p.err, kErrInvalidArg);
+    const int tile = blockIdx.x;
     const int bh = tile / n_kv;
-    // Causal heads are claimed from their last key block down: block j waits for block j+1.
-    const int j = p.causal ? (n_kv - 1 - tile % n_kv) : (tile % n_kv);
+    const int j = tile % n_kv;  // key block (causal: the heaviest, j = 0, first)
     const int b = bh / p.H;
-    const int L = seq_len(p, b, threadIdx.x == 0 && tile % n_kv == 0);
+    const int L = seq_len(p, b, threadIdx.x == 0 && j == 0);
     const int k0 = j * C::BN;
 
     if (k0 >= L) {
@@ -218,16 +288,15 @@ __global__ void __launch_bounds__(512, 1)
         }
         return;
     }
-    const int V = (L + C::BN - 1) / C::BN;  // key blocks holding at least one visible key
-    // Non-causal heads rotate their query-block order when all V key blocks of a head can be
-    // resident together (the rotated order waits in a cycle j -> j+1 -> ... -> V-1 -> 0).
-    const bool rotated = !p.causal && V <= p.resident_ctas;
+    // Causal: only query blocks from the diagonal on see this key block.  Non-causal: start
+    // at query block j and wrap, so the key blocks of a head add into different query
+    // blocks at any moment instead of all hammering the same accumulator lines.
     const int i_start = p.causal ? j : 0;
     const int n_it = n_q - i_start;
     auto q_block = [&](int it) {
         if (p.causal) return j + it;
-        if (rotated) { const int i = j + it; return i < n_q ? i : i - n_q; }
-        return it;
+        const int i = j + it;
+        return i < n_q ? i : i - n_q;
     };
 
     if (threadIdx.x == 0) {
@@ -243,12 +312,7 @@ __global__ void __launch_bounds__(512, 1)
         mbar_init(bar_dqfull, 1);
         mbar_init(bar_dqempty, 128);
         mbar_init(bar_done, 1);
-        mbar_init(&bar_go[0], 1);
-        mbar_init(&bar_go[1], 1);
-        mbar_init(&bar_added[0], 128);
-        mbar_init(&bar_added[1], 128);
         *abort_flag = 0;
-        *published = 0;
         fence_barrier_init();
     }
     if (warp == 8) {
@@ -270,53 +334,61 @@ __global__ void __launch_bounds__(512, 1)
         // ------------------------------------------------------------ dQ drain
         const int r = threadIdx.x - 384;                // TMEM lane
         const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
+        const float factor = head_bound_factor(p, bh);
+        // Named barriers have no timeout: every drain thread executes each of them, also after
+        // a failed wait (`ok` then only skips the work).
         bool ok = true;
         for (int it = 0; it < n_it; ++it) {
             const int q0 = q_block(it) * C::BM;
-            ok = mbar_wait(bar_dqfull, it & 1, p.timeout_ns, abort_flag);
-            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-            tc_fence_after();
-            uint32_t v[128];
-            constexpr int NV = (D == 128) ? 128 : 64;
+            // fixed-point scale of query q0 + r (rows past N: scale 0), shared by the drain
+            // warps; barrier 2 before the reads and again after the last read of the step
+            {
+                const int q = q0 + r;
+                s_scale[r] =
+                    q < p.N ? fixed_point_scale(p.dOnorm[(size_t)bh * p.N + q], factor) : 0.f;
+            }
+            named_barrier(2, 128);
+            const float* sc = s_scale;
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_dqfull, it & 1, p.timeout_ns, abort_flag));
+            if (ok) {
+                tc_fence_after();
+                constexpr int NV = (D == 128) ? 128 : 64;
+                uint32_t v[NV];
 #pragma unroll
-            for (int q = 0; q < NV / 32; ++q) tmem_ld32(tmem + lane_base + C::TM_B + 32 * q, v + 32 * q);
-            tmem_ld_wait();
+                for (int q = 0; q < NV / 32; ++q) tmem_ld32(tmem + lane_base + C::TM_B + 32 * q, v + 32 * q);
+                tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < NV / 32; ++q) reg_fence32(v + 32 * q);
-            tc_fence_before();
-            mbar_arrive(bar_dqempty);           // B may take the next dP^T
-            ok = mbar_wait(&bar_go[it & 1], (it >> 1) & 1, p.timeout_ns, abort_flag);
-            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-            const bool first = contribution_pos(q0 / C::BM, j, V, p.causal != 0, rotated) == 0;
-            float* acc = p.dq_acc + ((size_t)bh * p.N_pad + q0) * D;
-            if constexpr (D == 128) {
-                // dQ^T: lane = feature r, column = query e: a warp covers 32 consecutive
-                // features of one query row, one 128-byte line per instruction.
-                float* dst = acc + r;
-                if (first) {
+                for (int q = 0; q < NV / 32; ++q) reg_fence32(v + 32 * q);
+                tc_fence_before();
+                mbar_arrive(bar_dqempty);           // B may take the next dP^T
+                int* acc = p.dq_acc + ((size_t)bh * p.N_pad + q0) * D;
+                if constexpr (D == 128) {
+                    // dQ^T: lane = feature r, column = query e; a warp instruction covers 32
+                    // consecutive features of one query row: one 128-byte line.
 #pragma unroll
-                    for (int e = 0; e < 128; ++e) dst[(size_t)e * D] = __uint_as_float(v[e]);
+                    for (int e = 0; e < 128; ++e)
+                        red_add_s32(acc + (size_t)e * D + r, __float2int_rn(__uint_as_float(v[e]) * sc[e]));
                 } else {
+                    // dQ: lane = query r, 64 features.  Convert, transpose 32 x 32 through
+                    // shared memory, then a warp instruction covers 32 consecutive features of
+                    // one row.
+                    int* xp = reinterpret_cast<int*>(smem + C::SMEM_XPOSE) + (warp % 4) * 32 * 33;
+                    const float s_row = sc[r];
 #pragma unroll
-                    for (int e = 0; e < 128; ++e) red_add_f32(dst + (size_t)e * D, __uint_as_float(v[e]));
-                }
-            } else {
-                // dQ: lane = query r, 64 features.
-                float* dst = acc + (size_t)r * D;
-                if (first) {
+                    for (int c = 0; c < 2; ++c) {
 #pragma unroll
-                    for (int e = 0; e < 64; e += 4)
-                        *reinterpret_cast<float4*>(dst + e) =
-                            make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
-                                        __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 64; e += 4)
-                        red_add_v4(dst + e, __uint_as_float(v[e]), __uint_as_float(v[e + 1]),
-                                   __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+                        for (int e = 0; e < 32; ++e)
+                            xp[lane * 33 + e] = __float2int_rn(__uint_as_float(v[32 * c + e]) * s_row);
+                        __syncwarp();
+#pragma unroll 4
+                        for (int row = 0; row < 32; ++row)
+                            red_add_s32(acc + (size_t)((warp % 4) * 32 + row) * D + 32 * c + lane,
+                                        xp[row * 33 + lane]);
+                        __syncwarp();
+                    }
                 }
             }
-            mbar_arrive(&bar_added[it & 1]);    // the ordering thread publishes the count
+            named_barrier(2, 128);  // every read of s_scale done before the next step writes
         }
         if (!ok) fail();
     } else if (warp >= 8) {
@@ -350,47 +422,6 @@ __global__ void __launch_bounds__(512, 1)
         for (int t = max(0, it - C::QST); t < it; ++t)
             mbar_wait(&bar_qfull[t % C::QST], (t / C::QST) & 1, p.timeout_ns, abort_flag);
         mbar_wait(bar_kv, 0, p.timeout_ns, abort_flag);
-      } else if (warp == 10 && lane == 0) {
-        // ------------------------------------------------------------ dQ add ordering: turns
-        // Step it: wait until key block j is next to add into query block q_block(it) and say
-        // so on bar_go[it & 1].  Publishing is left to warp 11, so this thread never waits for
-        // this CTA's own adds: a turn only ever depends on earlier steps, here and in the
-        // other CTAs (no cycle).  Before step it it waits until warp 11 has passed step it-2,
-        // so no phase of the alternating barrier pairs can be lapped.
-        bool ok = true;
-        for (int it = 0; ok && it < n_it; ++it) {
-            const int i = q_block(it);
-            const int pos = contribution_pos(i, j, V, p.causal != 0, rotated);
-            const int* sem = p.sem + (size_t)bh * n_q + i;
-            const uint64_t t0 = globaltimer_ns();
-            while (it >= 2 && *published < it - 1) {
-                if (*abort_flag || globaltimer_ns() - t0 > p.timeout_ns) { ok = false; break; }
-            }
-            if (!ok) break;
-            if (pos > 0) {
-                while (ld_acquire_gpu(sem) != pos) {
-                    if (*abort_flag || globaltimer_ns() - t0 > p.timeout_ns) { ok = false; break; }
-                }
-                if (!ok) break;
-            }
-            mbar_arrive(&bar_go[it & 1]);
-        }
-        if (!ok) fail();
-      } else if (warp == 11 && lane == 0) {
-        // ------------------------------------------------------------ dQ add ordering: counts
-        // Once the drain has issued step it's adds (bar_added), make them visible at GPU scope
-        // and publish the count that lets the next key block add into that query block.
-        bool ok = true;
-        for (int it = 0; it < n_it; ++it) {
-            if (!(ok = mbar_wait(&bar_added[it & 1], (it >> 1) & 1, p.timeout_ns, abort_flag)))
-                break;
-            const int i = q_block(it);
-            fence_acq_rel_gpu();  // the drain's adds, acquired through bar_added
-            st_release_gpu(p.sem + (size_t)bh * n_q + i,
-                           contribution_pos(i, j, V, p.causal != 0, rotated) + 1);
-            *published = it + 1;
-        }
-        if (!ok) fail();
       } else if (warp == 8 && lane == 0) {
         // ------------------------------------------------------------ MMA issuer
         constexpr uint32_t idS = idesc_bf16(128, 128, false, false);  // S^T, dP^T
@@ -502,21 +533,21 @@ __global__ void __launch_bounds__(512, 1)
         store_vectors(0);
         named_barrier(1, 256);
 
+        // Named barriers have no timeout, so every thread executes every one of them, also
+        // after a failed (timed-out or aborted) wait; `ok` then only skips the work.
         bool ok = true;
         for (int it = 0; it < n_it; ++it) {
             const int i = q_block(it);
-            const int q0 = i * C::BM;
             const float* lse2 = s_lse2 + (it & 1) * C::BM + 64 * h;
             const float* Dv = s_D + (it & 1) * C::BM + 64 * h;
             if (it + 1 < n_it) load_vectors(it + 1);  // stored at the end of this iteration
             const bool diag = p.causal && (i == j);
 
             // ---------------- P phase
-            ok = mbar_wait(bar_sfull, it & 1, p.timeout_ns, abort_flag);
-            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-            tc_fence_after();
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_sfull, it & 1, p.timeout_ns, abort_flag));
             float P[64];
-            {
+            if (ok) {
+                tc_fence_after();
                 uint32_t sv[64];
                 tmem_ld32(tmem + lane_base + C::TM_A + 64 * h, sv);
                 tmem_ld32(tmem + lane_base + C::TM_A + 64 * h + 32, sv + 32);
@@ -537,33 +568,34 @@ __global__ void __launch_bounds__(512, 1)
                 }
             }
             named_barrier(1, 256);  // every S^T column read before P^T overwrites columns
-            {
+            if (ok) {
                 uint32_t pw[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) pw[e] = pack_bf16x2(P[2 * e], P[2 * e + 1]);
                 tmem_st32(tmem + lane_base + C::TM_A + 32 * h, pw);
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(bar_pfull);
             }
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(bar_pfull);
 
             // ---------------- dS phase
-            ok = mbar_wait(bar_dpfull, it & 1, p.timeout_ns, abort_flag);
-            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-            tc_fence_after();
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_dpfull, it & 1, p.timeout_ns, abort_flag));
             uint32_t dw[32];
+            if (ok) {
+                tc_fence_after();
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t dp[32];
-                tmem_ld32(tmem + lane_base + C::TM_B + 64 * h + 32 * half, dp);
-                tmem_ld_wait();
-                reg_fence32(dp);
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t dp[32];
+                    tmem_ld32(tmem + lane_base + C::TM_B + 64 * h + 32 * half, dp);
+                    tmem_ld_wait();
+                    reg_fence32(dp);
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const int ee = 32 * half + e;
-                    const float d0 = P[ee] * (__uint_as_float(dp[e]) - Dv[ee]);
-                    const float d1 = P[ee + 1] * (__uint_as_float(dp[e + 1]) - Dv[ee + 1]);
-                    dw[ee / 2] = pack_bf16x2(d0, d1);
+                    for (int e = 0; e < 32; e += 2) {
+                        const int ee = 32 * half + e;
+                        const float d0 = P[ee] * (__uint_as_float(dp[e]) - Dv[ee]);
+                        const float d1 = P[ee + 1] * (__uint_as_float(dp[e + 1]) - Dv[ee + 1]);
+                        dw[ee / 2] = pack_bf16x2(d0, d1);
+                    }
                 }
             }
             // Next block's lse / D into the other buffer: every thread has passed this
@@ -571,18 +603,19 @@ __global__ void __launch_bounds__(512, 1)
             // below orders these stores before the next iteration's reads.
             if (it + 1 < n_it) store_vectors(it + 1);
             named_barrier(1, 256);  // every dP^T column read before dS^T overwrites columns
-            tmem_st32(tmem + lane_base + C::TM_B + 32 * h, dw);
-            // dS^T row r, queries [64h, 64h+64) = one 128-byte row of query chunk h; 16-byte
-            // unit u sits at position u ^ (r % 8) (the 128-byte swizzle the MMA reads).
+            if (ok) {
+                tmem_st32(tmem + lane_base + C::TM_B + 32 * h, dw);
+                // dS^T row r, queries [64h, 64h+64) = one 128-byte row of query chunk h; 16-byte
+                // unit u sits at position u ^ (r % 8) (the 128-byte swizzle the MMA reads).
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                *reinterpret_cast<uint4*>(ds_row + ((u ^ sw) << 4)) =
-                    make_uint4(dw[4 * u], dw[4 * u + 1], dw[4 * u + 2], dw[4 * u + 3]);
-            tmem_st_wait();
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(bar_dsfull);
-
+                for (int u = 0; u < 8; ++u)
+                    *reinterpret_cast<uint4*>(ds_row + ((u ^ sw) << 4)) =
+                        make_uint4(dw[4 * u], dw[4 * u + 1], dw[4 * u + 2], dw[4 * u + 3]);
+                tmem_st_wait();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(bar_dsfull);
+            }
         }
 
         // ---------------- epilogue: dV (warpgroup 0) and dK * scale (warpgroup 1)
@@ -639,32 +672,18 @@ cudaError_t launch_bwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
         configured = true;
     }
     const int BH = p.B * p.H;
-    const int n_q = (p.N + C::BM - 1) / C::BM;
     const int n_kv = (p.N + C::BN - 1) / C::BN;
-    const int rows = BH * p.N;
-    const int n_sem = BH * n_q;
-    {
-        constexpr int TPR = D / 8;
-        const long long threads = (long long)rows * TPR;
-        const int blocks = (int)((threads + 255) / 256);
-        fa_bwd_pre_kernel<D><<<blocks, 256, 0, stream>>>(p, rows, n_sem);
-    }
+    const dim3 chunks(p.N_pad / 128, BH);
+    fa_bwd_pre_kernel<D><<<chunks, 256, 0, stream>>>(p);
     fa_bwd_kernel<D><<<BH * n_kv, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
-    {
-        const long long total8 = (long long)rows * D / 8;
-        const int blocks = (int)((total8 + 255) / 256);
-        fa_bwd_dq_kernel<D><<<blocks, 256, 0, stream>>>(p, total8);
-    }
+    fa_bwd_dq_kernel<D><<<chunks, 256, 0, stream>>>(p);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_bwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const CUtensorMap& tdq_acc, const BwdParams& p,
-                       int num_sms, cudaStream_t stream) {
-    (void)tdq_acc;
-    (void)num_sms;
+                       const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream) {
     if (d == 64) return launch_bwd_d<64>(tq, tk, tv, tdo, p, stream);
     return launch_bwd_d<128>(tq, tk, tv, tdo, p, stream);
 }

@@ -28,35 +28,32 @@ struct BwdParams {
     const void* o;         // bf16 [B, H, N, d]
     const void* dO;        // bf16 [B, H, N, d]
     const float* lse;      // fp32 [B, H, N]
+    const void* k;         // bf16 [B, H, N, d] (read by the preprocess kernel for its bound)
+    const void* v;         // bf16 [B, H, N, d]
     void* dq;              // bf16 out
     void* dk;              // bf16 out
     void* dv;              // bf16 out
-    float* Dvec;           // fp32 [B, H, N]   workspace
-    float* dq_acc;         // fp32 [B, H, N_pad, d] workspace
-    int* sem;              // int32 [B, H, N_pad / 128] workspace (ordered-reduction counters)
-    int* tile_counter;     // int32 [1] workspace
+    float* Dvec;           // fp32 [B, H, N]            workspace: rowsum(dO * O)
+    float* dOnorm;         // fp32 [B, H, N]            workspace: |dO_i|_2
+    float* headmax;        // fp32 [B, H, N_pad/128, 2] workspace: per-chunk max |v_j|_2, max |k_jl|
+    int* dq_acc;           // int32 [B, H, N_pad, d]    workspace: fixed-point dQ accumulator
     const int* seqlens;
     int* err;
     int B, H, N, N_pad;
     float scale;
     float scale_log2;
     int causal;
-    int resident_ctas;     // CTAs of the main kernel that can be resident at once (1 per SM)
     uint64_t timeout_ns;
 };
 
 // Tensor maps: a bf16 [B*H, N, d] tensor seen as 3-D (d, N, B*H), 128-byte swizzle,
 // box = 64 columns x `box_rows` rows; rows past N read as zeros.
 bool make_bf16_map(CUtensorMap* map, const void* base, int d, int N, int BH, int box_rows);
-// An fp32 [B*H, N_pad, d] tensor seen as 3-D (d, N_pad, B*H), 128-byte swizzle,
-// box = 32 columns x `box_rows` rows.
-bool make_f32_map(CUtensorMap* map, const void* base, int d, int N_pad, int BH, int box_rows);
 
 cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const FwdParams& p, int B, int num_sms, cudaStream_t stream);
 
 cudaError_t launch_bwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const CUtensorMap& tdq_acc, const BwdParams& p,
-                       int num_sms, cudaStream_t stream);
+                       const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream);
 
 }  // namespace fa

@@ -294,6 +294,10 @@ __device__ __forceinline__ void fence_acq_rel_gpu() {
 __device__ __forceinline__ void named_barrier_arrive(int id, int count) {
     asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
+// Integer add of one int32 into global memory (no return value).
+__device__ __forceinline__ void red_add_s32(int* p, int a) {
+    asm volatile("red.global.add.s32 [%0], %1;" ::"l"(p), "r"(a) : "memory");
+}
 // Named barrier over `count` threads (a multiple of 32) of this CTA.
 __device__ __forceinline__ void named_barrier(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");

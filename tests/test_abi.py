@@ -39,13 +39,13 @@ def test_status_strings():
 
 
 def test_workspace_size_formula():
-    # D (fp32 per row) + dQ accumulator (fp32, rows padded to 128) + counters + tile counter,
-    # each rounded up to 256 bytes.
+    # D and |dO_i| (fp32 per row), per-128-row-chunk maxima of |v_j| and |k_jl| (2 fp32), and
+    # the int32 fixed-point dQ accumulator (rows padded to 128), each rounded up to 256 bytes.
     def r(n):
         return (n + 255) // 256 * 256
     for B, H, N, d in ((1, 1, 1, 64), (2, 3, 300, 128), (4, 16, 4096, 128)):
         Np = (N + 127) // 128 * 128
-        expect = r(B * H * N * 4) + r(B * H * Np * d * 4) + r(B * H * (Np // 128) * 4) + r(4)
+        expect = 2 * r(B * H * N * 4) + r(B * H * (Np // 128) * 2 * 4) + r(B * H * Np * d * 4)
         assert fa.bwd_workspace_size(B, H, N, d) == expect
     assert fa.bwd_workspace_size(1, 1, 128, 96) == 0
     assert fa.bwd_workspace_size(0, 1, 128, 64) == 0
