@@ -124,6 +124,38 @@ FA_API fa_status fa_check_device_error(fa_stream_t stream);
  */
 FA_API void fa_set_wait_timeout_ns(uint64_t ns);
 
+/*
+ * fa_bwd_noalloc -- the backward pass without any device allocation.  The pages have no
+ * counterpart of this entry point; it exists for callers that cannot allocate device memory:
+ * a process that reserves its whole device-memory budget for its own pool up front, or a
+ * latency-critical loop that must not call cudaMalloc / cudaFree (they can block and
+ * synchronise the device).
+ *
+ * It computes exactly what fa_bwd computes, with the same kernels, arguments, layouts and
+ * results, but its scratch (the workspace fa_bwd takes from the caller) is a fixed area of
+ * FA_BWD_NOALLOC_SCRATCH_BYTES inside this library's own device code image: every GPU that
+ * loads the library holds that area until the process exits.  The caller still provides
+ * every input and output buffer.
+ *   error_flag  optional caller-owned device int (4-byte aligned): device-side errors of this
+ *               call (a bad sequence length, a wait that timed out) are stored there as an
+ *               fa_status code; it is never cleared by the library.  NULL: not reported.
+ * Limits and rules:
+ *   - Problems whose fa_bwd_workspace_size(B, H, N, d) exceeds FA_BWD_NOALLOC_SCRATCH_BYTES
+ *     are rejected with FA_ERR_WORKSPACE (e.g. B*H = 16, N = 4096, d = 128 fits;
+ *     B*H = 64 at the same N and d does not).
+ *   - All calls on a device share the one scratch area and each call overwrites it.  Calls
+ *     whose kernels overlap on the GPU (other streams, other host threads) race and give
+ *     wrong results: issue them on one stream, or order them yourself.
+ *   - The first call on a device performs a one-time set-up on the host (it looks up the
+ *     scratch area's device address); make that first call before any stream capture.
+ *   - No cudaMalloc, cudaFree or other allocating call is made, ever.
+ */
+#define FA_BWD_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+FA_API fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                                const void* dO, const float* lse, void* dq, void* dk, void* dv,
+                                int B, int H, int N, int d, float scale, int causal,
+                                const int* seqlens, int* error_flag, fa_stream_t stream);
+
 /* Static, human-readable name of a status code. */
 FA_API const char* fa_status_string(fa_status s);
 

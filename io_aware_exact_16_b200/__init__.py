@@ -44,7 +44,7 @@ _lib.fa_status_string.restype = ctypes.c_char_p
 
 # Every symbol include/fa.h declares.
 EXPORTED = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_check_device_error",
-            "fa_set_wait_timeout_ns", "fa_status_string")
+            "fa_set_wait_timeout_ns", "fa_status_string", "fa_bwd_noalloc")
 
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_WORKSPACE = range(6)
 

@@ -96,6 +96,8 @@ int pad128(int N) { return (N + 127) / 128 * 128; }
 
 }  // namespace
 
+uint64_t wait_timeout_ns() { return g_timeout_ns.load(); }
+
 bool make_bf16_map(CUtensorMap* map, const void* base, int d, int N, int BH, int box_rows) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;

@@ -46,6 +46,9 @@ struct BwdParams {
     uint64_t timeout_ns;
 };
 
+// Current bound on device-side waits (fa_set_wait_timeout_ns).
+uint64_t wait_timeout_ns();
+
 // Tensor maps: a bf16 [B*H, N, d] tensor seen as 3-D (d, N, B*H), 128-byte swizzle,
 // box = 64 columns x `box_rows` rows; rows past N read as zeros.
 bool make_bf16_map(CUtensorMap* map, const void* base, int d, int N, int BH, int box_rows);
