@@ -99,7 +99,7 @@ FA_API size_t fa_bwd_workspace_size(int B, int H, int N, int d);
  *   workspace      scratch of at least fa_bwd_workspace_size(B, H, N, d) bytes, 16-byte
  *                  aligned, owned by the caller, not used concurrently by another call.
  * The dQ sum over key blocks is exact integer (fixed-point) arithmetic: each key block's
- * contribution to query row i is rounded once to 2^-30 of an a-priori bound of row i
+ * contribution to query row i is rounded once to 2^-21 of an a-priori bound of row i
  * (2 |dO_i| max_j |v_j| max |k|) and the integer sum does not depend on the order in which
  * key blocks arrive, so repeated calls on the same inputs give bitwise identical dq, dk, dv.
  */

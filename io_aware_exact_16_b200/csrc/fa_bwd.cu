@@ -19,21 +19,23 @@
 // Deterministic dQ.  Every key block adds a contribution dS_ib K_b to every query row i it
 // sees.  Those contributions are added in integer fixed point, so the sum does not depend on
 // the order in which key blocks arrive and repeated runs are bitwise identical, with no
-// ordering between CTAs.  Row i uses the scale s_i = 2^floor(log2(2^30 / bound_i)), where
+// ordering between CTAs.  Row i uses the scale s_i = 2^floor(log2(2^21 / bound_i)), where
 //     bound_i = 2 |dO_i| max_j |v_j| max_{j,l} |k_jl|
 // bounds every partial sum: sum_j |dS_ij| = sum_j P_ij |dP_ij - D_i| <= 2 |dO_i| max_j |v_j|
 // (|dP_ij| <= |dO_i||v_j|, |D_i| <= |dO_i||O_i| and O_i is a convex combination of the v_j), and
-// each feature of sum_j dS_ij k_j is at most that times max |k_jl|.  Sums therefore stay below
-// 2^30 (+ one rounding per key block) and never overflow int32; each contribution is rounded
-// once, to 2^-30 bound_i.
+// each feature of sum_j dS_ij k_j is at most that times max |k_jl|.  Every contribution and
+// every partial sum therefore stays below 2^21 (+ one rounding per key block): far from int32
+// overflow, and below 2^22, where the rounding to an integer can run on the FMA pipe
+// (to_fixed).  Each contribution is rounded once, to 2^-21 bound_i.
 //
 // Main-kernel warp roles (512 threads = 4 warpgroups):
 //   warps 0-7   compute: warpgroup h owns query columns [64h, 64h+64) of every block; thread
 //               (h, r) owns key row r (= TMEM lane r).  Per query block two phases:
 //                 P   (needs S^T)  P^T = exp2(S^T c - lse2)   -> tensor memory (bf16)
 //                 dS  (needs dP^T) dS^T = P^T (dP^T - D)      -> tensor + shared memory (bf16)
-//               each overlapping one MMA (dP^T under P, dV under dS).  At the end they write
-//               dV (warpgroup 0) and dK (warpgroup 1).
+//               The MMA warp issues dV(i), S^T(i+1), dK(i), dQ(i), dP^T(i+1), so the P phase
+//               of block i+1 overlaps dK, dQ, the drain and dP^T of block i, and the dS phase
+//               overlaps dV and S^T.  At the end they write dV (warpgroup 0) and dK (wg 1).
 //   warp  8     MMA issue (one thread) + TMEM allocation
 //   warp  9     TMA producer (one thread)
 //   warps 10-11 idle
@@ -52,6 +54,12 @@
 // blocks (and for d = 64 the drain's transpose buffers).
 #include "fa_internal.h"
 #include "sm100.cuh"
+
+// Of every 4 pairs of probabilities, this many take their exponential on the FMA pipe
+// (exp2_fma2) and the rest on the MUFU unit.
+#ifndef FA_BWD_EXP2_FMA_OF_4
+#define FA_BWD_EXP2_FMA_OF_4 0
+#endif
 
 namespace fa {
 namespace {
@@ -84,8 +92,8 @@ struct BwdCfg {
     static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = SMEM_MISC + 16;  // tmem address, abort flag
     static constexpr int THREADS = 512;
-    // 2 x 160 (compute) + 56 (MMA / TMA) + 136 (drain) = 4 x 128 launched
-    static constexpr uint32_t REGS_COMPUTE = 160, REGS_OTHER = 56, REGS_DRAIN = 136;
+    // 2 x 136 (compute) + 88 (MMA / TMA) + 152 (drain) = 4 x 128 launched
+    static constexpr uint32_t REGS_COMPUTE = 136, REGS_OTHER = 88, REGS_DRAIN = 152;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t TM_A = 0, TM_B = 128, TM_DV = 256, TM_DK = 256 + D;
 };
@@ -119,14 +127,21 @@ __device__ __forceinline__ float head_bound_factor(const BwdParams& p, int bh) {
     return 2.0f * vmax * kmax;
 }
 
-// Fixed-point scale of a query row: the largest power of two s with s * bound <= 2^30;
+// Fixed-point scale of a query row: the largest power of two s with s * bound <= 2^21;
 // 0 when the bound is 0 (then every contribution of the row is 0).
 __device__ __forceinline__ float fixed_point_scale(float dO_norm, float head_factor) {
     const float bound = dO_norm * head_factor;
     if (!(bound > 0.f)) return 0.f;
-    const float x = 1073741824.0f / bound;
+    const float x = 2097152.0f / bound;
     if (!(x <= 3.0e38f)) return 0.f;
     return __int_as_float(__float_as_int(x) & 0x7F800000);  // 2^floor(log2 x), exact
+}
+
+// round(v * s) as an integer for |v * s| < 2^22, on the FMA pipe: adding 1.5 * 2^23 leaves
+// the rounded value in the low mantissa bits (ties to even), which the integer subtraction
+// reads out.  (The conversion instruction would run on the unit the exponentials need.)
+__device__ __forceinline__ int to_fixed(float v, float s) {
+    return __float_as_int(fmaf(v, s, 12582912.0f)) - 0x4B400000;
 }
 
 // ---------------------------------------------------------------------------- preprocess
@@ -367,7 +382,7 @@ __global__ void __launch_bounds__(512, 1)
                     // consecutive features of one query row: one 128-byte line.
 #pragma unroll
                     for (int e = 0; e < 128; ++e)
-                        red_add_s32(acc + (size_t)e * D + r, __float2int_rn(__uint_as_float(v[e]) * sc[e]));
+                        red_add_s32(acc + (size_t)e * D + r, to_fixed(__uint_as_float(v[e]), sc[e]));
                 } else {
                     // dQ: lane = query r, 64 features.  Convert, transpose 32 x 32 through
                     // shared memory, then a warp instruction covers 32 consecutive features of
@@ -378,7 +393,7 @@ __global__ void __launch_bounds__(512, 1)
                     for (int c = 0; c < 2; ++c) {
 #pragma unroll
                         for (int e = 0; e < 32; ++e)
-                            xp[lane * 33 + e] = __float2int_rn(__uint_as_float(v[32 * c + e]) * s_row);
+                            xp[lane * 33 + e] = to_fixed(__uint_as_float(v[32 * c + e]), s_row);
                         __syncwarp();
 #pragma unroll 4
                         for (int row = 0; row < 32; ++row)
@@ -427,55 +442,70 @@ __global__ void __launch_bounds__(512, 1)
         constexpr uint32_t idS = idesc_bf16(128, 128, false, false);  // S^T, dP^T
         constexpr uint32_t idKV = idesc_bf16(128, D, false, true);    // dV, dK (A in TMEM)
         constexpr uint32_t idQ = idesc_bf16(128, D == 128 ? 128 : 64, true, true);  // dQ^T / dQ
-        const uint32_t sK = smem_u32(smem + C::SMEM_K);
-        const uint32_t sV = smem_u32(smem + C::SMEM_V);
-        const uint32_t sQ = smem_u32(smem + C::SMEM_Q);
-        const uint32_t sDO = smem_u32(smem + C::SMEM_DO);
-        const uint32_t sDS = smem_u32(smem + C::SMEM_DS);
+        // Descriptors of every operand tile, built once; a K step only adds the byte offset
+        // (>> 4) to the start-address field, which never carries (shared memory < 256 KB).
+        const uint64_t dK_k = sdesc_sw128(smem_u32(smem + C::SMEM_K), 16, 1024);   // K-major
+        const uint64_t dV_k = sdesc_sw128(smem_u32(smem + C::SMEM_V), 16, 1024);
+        const uint64_t dK_mn = sdesc_sw128(smem_u32(smem + C::SMEM_K), C::CHUNK_BYTES, 1024);
+        const uint64_t dDS_mn = sdesc_sw128(smem_u32(smem + C::SMEM_DS), C::CHUNK_BYTES, 1024);
+        // Q / dO stage st sits st * Q_TILE_BYTES after stage 0.
+        const uint64_t dQ_k0 = sdesc_sw128(smem_u32(smem + C::SMEM_Q), 16, 1024);
+        const uint64_t dDO_k0 = sdesc_sw128(smem_u32(smem + C::SMEM_DO), 16, 1024);
+        const uint64_t dQ_mn0 = sdesc_sw128(smem_u32(smem + C::SMEM_Q), C::CHUNK_BYTES, 1024);
+        const uint64_t dDO_mn0 = sdesc_sw128(smem_u32(smem + C::SMEM_DO), C::CHUNK_BYTES, 1024);
+        auto kmaj = [](int kk) { return (uint64_t)(((kk / 4) * C::CHUNK_BYTES + (kk % 4) * 32) >> 4); };
+        auto mnmaj = [](int kk) { return (uint64_t)((kk * 2048) >> 4); };
+        auto stage_off = [](int it) { return (uint64_t)((it % C::QST) * (C::Q_TILE_BYTES >> 4)); };
+        // S^T = K Q^T and dP^T = V dO^T for query step `it`: K-major operands, 16-column K
+        // steps (32 bytes inside a swizzled row, then the next 64-column chunk).
+        auto issue_S = [&](int it) {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+                mma_ss(tmem + C::TM_A, dK_k + kmaj(kk), dQ_k0 + stage_off(it) + kmaj(kk), idS,
+                       kk > 0 ? 1u : 0u);
+            tc_commit(bar_sfull);
+        };
+        auto issue_dP = [&](int it) {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+                mma_ss(tmem + C::TM_B, dV_k + kmaj(kk), dDO_k0 + stage_off(it) + kmaj(kk), idS,
+                       kk > 0 ? 1u : 0u);
+            tc_commit(bar_dpfull);
+        };
+        // Issue order per query step it:  dV(it), S^T(it+1), dK(it), dQ(it), dP^T(it+1).
+        // S^T(it+1) may go as soon as dV(it) has read P^T(it) from A (MMAs of one thread run
+        // in order), so the next P phase overlaps dK, dQ, the drain and dP^T.
         bool ok = mbar_wait(bar_kv, 0, p.timeout_ns, abort_flag);
+        if (ok) ok = mbar_wait(&bar_qfull[0], 0, p.timeout_ns, abort_flag);
+        if (ok) {
+            tc_fence_after();
+            issue_S(0);
+            issue_dP(0);
+        }
         for (int it = 0; ok && it < n_it; ++it) {
             const int s = it % C::QST;
-            const uint32_t ph = (it / C::QST) & 1;
-            const uint32_t qa = sQ + s * C::Q_TILE_BYTES;
-            const uint32_t da = sDO + s * C::Q_TILE_BYTES;
-            if (!(ok = mbar_wait(&bar_qfull[s], ph, p.timeout_ns, abort_flag))) break;
-            tc_fence_after();
-            // S^T = K Q^T: K-major operands, 16-column K steps (32 bytes inside a swizzled row,
-            // then the next 64-column chunk).
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk / 4) * C::CHUNK_BYTES + (kk % 4) * 32;
-                mma_ss(tmem + C::TM_A, sdesc_sw128(sK + off, 16, 1024),
-                       sdesc_sw128(qa + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
-            }
-            tc_commit(bar_sfull);
-            // dP^T = V dO^T into B, once the previous dQ block has been drained from B.
-            if (it > 0 && !(ok = mbar_wait(bar_dqempty, (it - 1) & 1, p.timeout_ns, abort_flag)))
-                break;
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk / 4) * C::CHUNK_BYTES + (kk % 4) * 32;
-                mma_ss(tmem + C::TM_B, sdesc_sw128(sV + off, 16, 1024),
-                       sdesc_sw128(da + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
-            }
-            tc_commit(bar_dpfull);
+            const uint64_t dQ_mn = dQ_mn0 + stage_off(it), dDO_mn = dDO_mn0 + stage_off(it);
             // dV += P^T dO: A = P^T in tensor memory (16 queries = 8 columns per K step),
             // B = dO MN-major (16 query rows = 2048 bytes per K step).
             if (!(ok = mbar_wait(bar_pfull, it & 1, p.timeout_ns, abort_flag))) break;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < C::BM / 16; ++kk)
-                mma_ts(tmem + C::TM_DV, tmem + C::TM_A + kk * 8,
-                       sdesc_sw128(da + kk * 2048, C::CHUNK_BYTES, 1024), idKV,
+                mma_ts(tmem + C::TM_DV, tmem + C::TM_A + kk * 8, dDO_mn + mnmaj(kk), idKV,
                        (it > 0 || kk > 0) ? 1u : 0u);
-            // dK += dS^T Q, same shapes.
+            if (it + 1 < n_it) {
+                const int s1 = (it + 1) % C::QST;
+                if (!(ok = mbar_wait(&bar_qfull[s1], ((it + 1) / C::QST) & 1, p.timeout_ns, abort_flag)))
+                    break;
+                tc_fence_after();
+                issue_S(it + 1);
+            }
+            // dK += dS^T Q, same shapes as dV.
             if (!(ok = mbar_wait(bar_dsfull, it & 1, p.timeout_ns, abort_flag))) break;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < C::BM / 16; ++kk)
-                mma_ts(tmem + C::TM_DK, tmem + C::TM_B + kk * 8,
-                       sdesc_sw128(qa + kk * 2048, C::CHUNK_BYTES, 1024), idKV,
+                mma_ts(tmem + C::TM_DK, tmem + C::TM_B + kk * 8, dQ_mn + mnmaj(kk), idKV,
                        (it > 0 || kk > 0) ? 1u : 0u);
             tc_commit(&bar_qempty[s]);
             // The dQ block into B; K steps of 16 keys = 2048 bytes of both tiles, both
@@ -484,18 +514,22 @@ __global__ void __launch_bounds__(512, 1)
                 // dQ^T = K^T dS^T: A = K^T (M = feature), B = dS^T (N = query).
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 16; ++kk)
-                    mma_ss(tmem + C::TM_B, sdesc_sw128(sK + kk * 2048, C::CHUNK_BYTES, 1024),
-                           sdesc_sw128(sDS + kk * 2048, C::CHUNK_BYTES, 1024), idQ,
+                    mma_ss(tmem + C::TM_B, dK_mn + mnmaj(kk), dDS_mn + mnmaj(kk), idQ,
                            kk > 0 ? 1u : 0u);
             } else {
                 // dQ = dS K: A = dS (M = query, from the dS^T tile), B = K (N = feature).
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 16; ++kk)
-                    mma_ss(tmem + C::TM_B, sdesc_sw128(sDS + kk * 2048, C::CHUNK_BYTES, 1024),
-                           sdesc_sw128(sK + kk * 2048, C::CHUNK_BYTES, 1024), idQ,
+                    mma_ss(tmem + C::TM_B, dDS_mn + mnmaj(kk), dK_mn + mnmaj(kk), idQ,
                            kk > 0 ? 1u : 0u);
             }
             tc_commit(bar_dqfull);
+            // dP^T(it+1) into B once the drain has copied the dQ block out.
+            if (it + 1 < n_it) {
+                if (!(ok = mbar_wait(bar_dqempty, it & 1, p.timeout_ns, abort_flag))) break;
+                tc_fence_after();
+                issue_dP(it + 1);
+            }
         }
         if (!ok) fail();
         // Wait for every MMA issued here before tensor memory can be released.
@@ -515,14 +549,14 @@ __global__ void __launch_bounds__(512, 1)
         const int sw = r & 7;
         const float c = p.scale_log2;
 
-        // lse * log2(e) and D of query block q_block(it) into buffer it & 1 (threads 0..127 the
-        // lse values, 128..255 the D values); +inf / 0 past N so those queries get P = 0.
+        // -lse * log2(e) and D of query block q_block(it) into buffer it & 1 (threads 0..127 the
+        // lse values, 128..255 the D values); -inf / 0 past N so those queries get P = 0.
         // The global load is issued one iteration ahead (load_vectors) and stored to shared
         // memory at the end of the iteration (store_vectors), so its latency stays hidden.
         float staged = 0.f;
         auto load_vectors = [&](int it) {
             const int q = q_block(it) * C::BM + (ct & 127);
-            if (ct < 128) staged = q < p.N ? p.lse[(size_t)bh * p.N + q] * kLog2e : INFINITY;
+            if (ct < 128) staged = q < p.N ? -p.lse[(size_t)bh * p.N + q] * kLog2e : -INFINITY;
             else staged = q < p.N ? p.Dvec[(size_t)bh * p.N + q] : 0.f;
         };
         auto store_vectors = [&](int it) {
@@ -555,11 +589,20 @@ __global__ void __launch_bounds__(512, 1)
                 reg_fence32(sv);
                 reg_fence32(sv + 32);
 #pragma unroll
-                for (int e = 0; e < 64; e += 2) {
-                    const float2 x = ffma2(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])),
-                                           make_float2(c, c), make_float2(-lse2[e], -lse2[e + 1]));
-                    P[e] = ex2(x.x);
-                    P[e + 1] = ex2(x.y);
+                for (int e = 0; e < 64; e += 4) {
+                    const float4 nl = *reinterpret_cast<const float4*>(lse2 + e);  // -lse2
+#pragma unroll
+                    for (int u = 0; u < 4; u += 2) {
+                        const float2 x = ffma2(make_float2(__uint_as_float(sv[e + u]),
+                                                           __uint_as_float(sv[e + u + 1])),
+                                               make_float2(c, c),
+                                               u == 0 ? make_float2(nl.x, nl.y) : make_float2(nl.z, nl.w));
+                        const float2 pe = (((e + u) / 2) % 4 < FA_BWD_EXP2_FMA_OF_4)
+                                              ? exp2_fma2(x)
+                                              : make_float2(ex2(x.x), ex2(x.y));
+                        P[e + u] = pe.x;
+                        P[e + u + 1] = pe.y;
+                    }
                 }
                 if (key_padded || diag) {
 #pragma unroll
@@ -590,11 +633,17 @@ __global__ void __launch_bounds__(512, 1)
                     tmem_ld_wait();
                     reg_fence32(dp);
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
+                    for (int e = 0; e < 32; e += 4) {
                         const int ee = 32 * half + e;
-                        const float d0 = P[ee] * (__uint_as_float(dp[e]) - Dv[ee]);
-                        const float d1 = P[ee + 1] * (__uint_as_float(dp[e + 1]) - Dv[ee + 1]);
-                        dw[ee / 2] = pack_bf16x2(d0, d1);
+                        const float4 dv4 = *reinterpret_cast<const float4*>(Dv + ee);
+                        const float2 a = fmul2(make_float2(P[ee], P[ee + 1]),
+                                               fadd2(make_float2(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])),
+                                                     make_float2(-dv4.x, -dv4.y)));
+                        const float2 b = fmul2(make_float2(P[ee + 2], P[ee + 3]),
+                                               fadd2(make_float2(__uint_as_float(dp[e + 2]), __uint_as_float(dp[e + 3])),
+                                                     make_float2(-dv4.z, -dv4.w)));
+                        dw[ee / 2] = pack_bf16x2(a.x, a.y);
+                        dw[ee / 2 + 1] = pack_bf16x2(b.x, b.y);
                     }
                 }
             }

@@ -31,6 +31,12 @@
 #include "fa_internal.h"
 #include "sm100.cuh"
 
+// Of every 4 pairs of scores, this many take their exponential on the FMA pipe (exp2_fma2)
+// and the rest on the MUFU unit, so the two units share the softmax's exponentials.
+#ifndef FA_FWD_EXP2_FMA_OF_4
+#define FA_FWD_EXP2_FMA_OF_4 0
+#endif
+
 namespace fa {
 namespace {
 
@@ -333,7 +339,9 @@ __global__ void __launch_bounds__(384, 1)
                     const int e0 = h * 64 + 2 * i;
                     const float2 x = ffma2(make_float2(__uint_as_float(s[e0]),
                                                        __uint_as_float(s[e0 + 1])), c2, nm2);
-                    const float2 e = make_float2(ex2(x.x), ex2(x.y));
+                    const float2 e = (i % 4 < FA_FWD_EXP2_FMA_OF_4)
+                                         ? exp2_fma2(x)
+                                         : make_float2(ex2(x.x), ex2(x.y));
                     acc[i % 4] = fadd2(acc[i % 4], e);
                     pk[i] = pack_bf16x2(e.x, e.y);
                 }
