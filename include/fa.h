@@ -125,6 +125,25 @@ FA_API fa_status fa_check_device_error(fa_stream_t stream);
 FA_API void fa_set_wait_timeout_ns(uint64_t ns);
 
 /*
+ * Grouped-query / multi-query attention (FlashAttention (DE), section on FlashAttention-2:
+ * support for multi-query attention).  Same as fa_fwd / fa_bwd, except that K and V (and dK,
+ * dV) have H_kv heads, [B, H_kv, N, d], with H % H_kv == 0: query head h attends with key/value
+ * head h / (H / H_kv) (consecutive query heads share one key/value head; H_kv = 1 is
+ * multi-query attention, H_kv = H is fa_fwd / fa_bwd).  dK and dV of a key/value head are the
+ * sums over its query heads, formed inside one CTA in a fixed order (no atomics), so repeated
+ * calls stay bitwise identical.  The workspace is fa_bwd_workspace_size(B, H, N, d) (query
+ * heads).  H_kv outside [1, H] or not dividing H: FA_ERR_INVALID_ARG.
+ */
+FA_API fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
+                            int B, int H, int H_kv, int N, int d, float scale, int causal,
+                            const int* seqlens, fa_stream_t stream);
+FA_API fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
+                            const void* dO, const float* lse, void* dq, void* dk, void* dv,
+                            int B, int H, int H_kv, int N, int d, float scale, int causal,
+                            const int* seqlens, void* workspace, size_t workspace_bytes,
+                            fa_stream_t stream);
+
+/*
  * fa_bwd_noalloc -- the backward pass without any device allocation.  The pages have no
  * counterpart of this entry point; it exists for callers that cannot allocate device memory:
  * a process that reserves its whole device-memory budget for its own pool up front, or a

@@ -33,6 +33,12 @@ _lib.fa_fwd.restype = _i
 _lib.fa_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
                         ctypes.c_float, _i, _vp, _vp, ctypes.c_size_t, _vp]
 _lib.fa_bwd.restype = _i
+_lib.fa_fwd_gqa.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float, _i, _vp,
+                            _vp]
+_lib.fa_fwd_gqa.restype = _i
+_lib.fa_bwd_gqa.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
+                            ctypes.c_float, _i, _vp, _vp, ctypes.c_size_t, _vp]
+_lib.fa_bwd_gqa.restype = _i
 _lib.fa_bwd_workspace_size.argtypes = [_i, _i, _i, _i]
 _lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
 _lib.fa_check_device_error.argtypes = [_vp]
@@ -43,8 +49,9 @@ _lib.fa_status_string.argtypes = [_i]
 _lib.fa_status_string.restype = ctypes.c_char_p
 
 # Every symbol include/fa.h declares.
-EXPORTED = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_check_device_error",
-            "fa_set_wait_timeout_ns", "fa_status_string", "fa_bwd_noalloc")
+EXPORTED = ("fa_fwd", "fa_bwd", "fa_fwd_gqa", "fa_bwd_gqa", "fa_bwd_workspace_size",
+            "fa_check_device_error", "fa_set_wait_timeout_ns", "fa_status_string",
+            "fa_bwd_noalloc")
 
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_WORKSPACE = range(6)
 
@@ -86,14 +93,28 @@ def _seqlens_ptr(seqlens: Optional[torch.Tensor], B: int, device) -> int:
     return seqlens.data_ptr()
 
 
+def _kv_heads(q: torch.Tensor, k: torch.Tensor) -> int:
+    """Key/value heads of k ([B, H_kv, N, d]); H_kv must divide q's H (grouped-query attention)."""
+    if k.dim() != 4:
+        raise ValueError(f"k must be [B, H_kv, N, d], got shape {tuple(k.shape)}")
+    H, H_kv = q.shape[1], k.shape[1]
+    if H_kv < 1 or H % H_kv != 0:
+        raise ValueError(f"key/value heads {H_kv} must divide query heads {H}")
+    return H_kv
+
+
 def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
             seqlens: Optional[torch.Tensor] = None, scale: Optional[float] = None,
             out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None):
-    """``fa_fwd``: returns (O bf16 [B, H, N, d], lse fp32 [B, H, N]) on q's device/stream."""
+    """``fa_fwd_gqa`` (``fa_fwd`` when k, v have as many heads as q): returns
+    (O bf16 [B, H, N, d], lse fp32 [B, H, N]) on q's device and current stream.
+    k and v may have fewer heads, [B, H_kv, N, d] with H % H_kv == 0."""
     B, H, N, d = q.shape
     dev = q.device
-    for name, t in (("q", q), ("k", k), ("v", v)):
-        _check_qkv(name, t, (B, H, N, d), dev)
+    H_kv = _kv_heads(q, k)
+    _check_qkv("q", q, (B, H, N, d), dev)
+    for name, t in (("k", k), ("v", v)):
+        _check_qkv(name, t, (B, H_kv, N, d), dev)
     if out is None:
         out = torch.empty_like(q)
     else:
@@ -103,11 +124,11 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = Fa
     elif lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous float32 tensor [B, H, N]")
     sc = float(scale) if scale is not None else 1.0 / (d ** 0.5)
-    st = _lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                     B, H, N, d, sc, int(bool(causal)), _seqlens_ptr(seqlens, B, dev),
-                     _stream_handle(dev))
+    st = _lib.fa_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                         B, H, H_kv, N, d, sc, int(bool(causal)), _seqlens_ptr(seqlens, B, dev),
+                         _stream_handle(dev))
     if st != FA_OK:
-        raise FAError(st, "fa_fwd")
+        raise FAError(st, "fa_fwd_gqa")
     return out, lse
 
 
@@ -118,28 +139,34 @@ def bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
 def backward(q, k, v, o, do, lse, causal: bool = False, seqlens: Optional[torch.Tensor] = None,
              scale: Optional[float] = None, dq=None, dk=None, dv=None,
              workspace: Optional[torch.Tensor] = None):
-    """``fa_bwd``: returns (dQ, dK, dV), bf16 [B, H, N, d]."""
+    """``fa_bwd_gqa`` (``fa_bwd`` when k, v have as many heads as q): returns (dQ, dK, dV) in
+    bf16, dK and dV shaped like k and v."""
     B, H, N, d = q.shape
     dev = q.device
-    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
+    H_kv = _kv_heads(q, k)
+    for name, t in (("q", q), ("o", o), ("do", do)):
         _check_qkv(name, t, (B, H, N, d), dev)
+    for name, t in (("k", k), ("v", v)):
+        _check_qkv(name, t, (B, H_kv, N, d), dev)
     if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous float32 tensor [B, H, N]")
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
-        _check_qkv(name, t, (B, H, N, d), dev)
+    _check_qkv("dq", dq, (B, H, N, d), dev)
+    for name, t in (("dk", dk), ("dv", dv)):
+        _check_qkv(name, t, (B, H_kv, N, d), dev)
     need = bwd_workspace_size(B, H, N, d)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
     sc = float(scale) if scale is not None else 1.0 / (d ** 0.5)
-    st = _lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
-                     lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, sc,
-                     int(bool(causal)), _seqlens_ptr(seqlens, B, dev), workspace.data_ptr(),
-                     workspace.numel() * workspace.element_size(), _stream_handle(dev))
+    st = _lib.fa_bwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                         lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, H_kv,
+                         N, d, sc, int(bool(causal)), _seqlens_ptr(seqlens, B, dev),
+                         workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                         _stream_handle(dev))
     if st != FA_OK:
-        raise FAError(st, "fa_bwd")
+        raise FAError(st, "fa_bwd_gqa")
     return dq, dk, dv
 
 

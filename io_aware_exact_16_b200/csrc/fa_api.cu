@@ -132,10 +132,12 @@ void fa_set_wait_timeout_ns(uint64_t ns) {
     g_timeout_ns.store(ns < 1000000ull ? 1000000ull : ns);
 }
 
-fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-                 int N, int d, float scale, int causal, const int* seqlens, fa_stream_t stream) {
+fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int H, int H_kv, int N, int d, float scale, int causal, const int* seqlens,
+                     fa_stream_t stream) {
     fa_status st = check_common(B, H, N, d, scale);
     if (st != FA_OK) return st;
+    if (H_kv < 1 || H_kv > H || H % H_kv != 0) return FA_ERR_INVALID_ARG;
     if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
         return FA_ERR_INVALID_ARG;
@@ -144,8 +146,8 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     if (!dev) return st;
 
     CUtensorMap tq, tk, tv;
-    if (!make_bf16_map(&tq, q, d, N, B * H, 128) || !make_bf16_map(&tk, k, d, N, B * H, 128) ||
-        !make_bf16_map(&tv, v, d, N, B * H, 128))
+    if (!make_bf16_map(&tq, q, d, N, B * H, 128) || !make_bf16_map(&tk, k, d, N, B * H_kv, 128) ||
+        !make_bf16_map(&tv, v, d, N, B * H_kv, 128))
         return FA_ERR_CUDA;
     FwdParams p{};
     p.o = o;
@@ -154,6 +156,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     p.err = dev->err_flag;
     p.H = H;
     p.N = N;
+    p.H_kv = H_kv;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
     p.timeout_ns = g_timeout_ns.load();
@@ -161,6 +164,11 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
         cudaSuccess)
         return FA_ERR_CUDA;
     return FA_OK;
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int N, int d, float scale, int causal, const int* seqlens, fa_stream_t stream) {
+    return fa_fwd_gqa(q, k, v, o, lse, B, H, H, N, d, scale, causal, seqlens, stream);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
@@ -176,12 +184,13 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
     return bytes;
 }
 
-fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
-                 const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
-                 float scale, int causal, const int* seqlens, void* workspace,
-                 size_t workspace_bytes, fa_stream_t stream) {
+fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
+                     const void* dO, const float* lse, void* dq, void* dk, void* dv, int B, int H,
+                     int H_kv, int N, int d, float scale, int causal, const int* seqlens,
+                     void* workspace, size_t workspace_bytes, fa_stream_t stream) {
     fa_status st = check_common(B, H, N, d, scale);
     if (st != FA_OK) return st;
+    if (H_kv < 1 || H_kv > H || H % H_kv != 0) return FA_ERR_INVALID_ARG;
     if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dO) ||
         !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
@@ -220,18 +229,27 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
     p.H = H;
     p.N = N;
     p.N_pad = Np;
+    p.H_kv = H_kv;
     p.scale = scale;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
     p.timeout_ns = g_timeout_ns.load();
 
     CUtensorMap tq, tk, tv, tdo;
-    if (!make_bf16_map(&tq, q, d, N, BH, 128) || !make_bf16_map(&tk, k, d, N, BH, 128) ||
-        !make_bf16_map(&tv, v, d, N, BH, 128) || !make_bf16_map(&tdo, dO, d, N, BH, 128))
+    if (!make_bf16_map(&tq, q, d, N, BH, 128) || !make_bf16_map(&tk, k, d, N, B * H_kv, 128) ||
+        !make_bf16_map(&tv, v, d, N, B * H_kv, 128) || !make_bf16_map(&tdo, dO, d, N, BH, 128))
         return FA_ERR_CUDA;
     if (launch_bwd(d, tq, tk, tv, tdo, p, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
         return FA_ERR_CUDA;
     return FA_OK;
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                 const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                 float scale, int causal, const int* seqlens, void* workspace,
+                 size_t workspace_bytes, fa_stream_t stream) {
+    return fa_bwd_gqa(q, k, v, o, dO, lse, dq, dk, dv, B, H, H, N, d, scale, causal, seqlens,
+                      workspace, workspace_bytes, stream);
 }
 
 fa_status fa_check_device_error(fa_stream_t stream) {

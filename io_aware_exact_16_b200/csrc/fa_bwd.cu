@@ -145,18 +145,20 @@ __device__ __forceinline__ int to_fixed(float v, float s) {
 }
 
 // ---------------------------------------------------------------------------- preprocess
-// Grid (N_pad / 128 chunks, B*H).  Per row: D = dO . O (fp32) and |dO|; per chunk: the largest
-// |v_j| and |k_jl| of its visible key rows (j < L_b); and the chunk's rows of the dQ
-// accumulator set to zero.  TPR threads per row, each reading 16 bytes of every tensor.
+// Grid (N_pad / 128 chunks, B*H).  Per query row: D = dO . O (fp32) and |dO|; per chunk of
+// key/value head (blocks y < B*H_kv): the largest |v_j| and |k_jl| of its visible key rows
+// (j < L_b); and the chunk's rows of the dQ accumulator set to zero.  TPR threads per row, each reading 16 bytes of every tensor.
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p) {
     constexpr int TPR = D / 8;               // threads per row
     constexpr int RPP = 256 / TPR;           // rows per pass
     const int chunk = blockIdx.x;
-    const int bh = blockIdx.y;
+    const int bh = blockIdx.y;                       // query head (b, h)
     const int part = threadIdx.x % TPR;
-    // Only keys some query can see enter the bound (padded keys contribute nothing to dQ).
-    const int L = seq_len(p, bh / p.H, false);
+    // Blocks of the first B * H_kv heads also scan key/value head bh for the bound maxima; only
+    // keys some query can see enter them (padded keys contribute nothing to dQ).
+    const bool kv_head = bh < p.B * p.H_kv;
+    const int L = kv_head ? seq_len(p, bh / p.H_kv, false) : 0;
     float vmax = 0.f, kmax = 0.f;
     for (int rr = threadIdx.x / TPR; rr < 128; rr += RPP) {
         const int n = chunk * 128 + rr;
@@ -165,20 +167,26 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p) {
             const size_t off = ((size_t)bh * p.N + n) * TPR + part;
             const uint4 a = reinterpret_cast<const uint4*>(p.dO)[off];
             const uint4 o = reinterpret_cast<const uint4*>(p.o)[off];
-            const uint4 v = reinterpret_cast<const uint4*>(p.v)[off];
-            const uint4 k = reinterpret_cast<const uint4*>(p.k)[off];
             const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
             const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&o);
-            const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&v);
-            const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&k);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const float2 fa = __bfloat1622float2(a2[i]);
                 const float2 fo = __bfloat1622float2(o2[i]);
-                const float2 fv = __bfloat1622float2(v2[i]);
-                const float2 fk = __bfloat1622float2(k2[i]);
                 dd = fmaf(fa.x, fo.x, fmaf(fa.y, fo.y, dd));
                 nn = fmaf(fa.x, fa.x, fmaf(fa.y, fa.y, nn));
+            }
+        }
+        if (n < L) {
+            const size_t off = ((size_t)bh * p.N + n) * TPR + part;
+            const uint4 v = reinterpret_cast<const uint4*>(p.v)[off];
+            const uint4 k = reinterpret_cast<const uint4*>(p.k)[off];
+            const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+            const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&k);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 fv = __bfloat1622float2(v2[i]);
+                const float2 fk = __bfloat1622float2(k2[i]);
                 vv = fmaf(fv.x, fv.x, fmaf(fv.y, fv.y, vv));
                 ka = fmaxf(ka, fmaxf(fabsf(fk.x), fabsf(fk.y)));
             }
@@ -194,10 +202,8 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p) {
             p.Dvec[(size_t)bh * p.N + n] = dd;
             p.dOnorm[(size_t)bh * p.N + n] = sqrtf(nn);
         }
-        if (n < L) {
-            vmax = fmaxf(vmax, sqrtf(vv));
-            kmax = fmaxf(kmax, ka);
-        }
+        vmax = fmaxf(vmax, sqrtf(vv));
+        kmax = fmaxf(kmax, ka);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
@@ -213,7 +219,7 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p) {
     int4* acc = reinterpret_cast<int4*>(p.dq_acc + ((size_t)bh * p.N_pad + (size_t)chunk * 128) * D);
     for (int i = threadIdx.x; i < 128 * D / 4; i += 256) acc[i] = make_int4(0, 0, 0, 0);
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && kv_head) {
         float a = 0.f, b = 0.f;
         for (int w = 0; w < 8; ++w) {
             a = fmaxf(a, red[0][w]);
@@ -232,7 +238,8 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const BwdParams p) {
     const int chunk = blockIdx.x;
     const int bh = blockIdx.y;
     __shared__ float s_factor;
-    if (threadIdx.x == 0) s_factor = head_bound_factor(p, bh);
+    if (threadIdx.x == 0)
+        s_factor = head_bound_factor(p, (bh / p.H) * p.H_kv + (bh % p.H) / (p.H / p.H_kv));
     __syncthreads();
     const float factor = s_factor;
     constexpr int PER_ROW = D / 8;  // 8 elements per thread-step
@@ -286,17 +293,19 @@ __global__ void __launch_bounds__(512, 1)
 
     if (threadIdx.x == 0 && (smem_u32(smem) & 1023u)) record_error(p.err, kErrInvalidArg);
     const int tile = blockIdx.x;
-    const int bh = tile / n_kv;
-    const int j = tile % n_kv;  // key block (causal: the heaviest, j = 0, first)
-    const int b = bh / p.H;
+    const int bhk = tile / n_kv;  // (batch, key/value head)
+    const int j = tile % n_kv;    // key block (causal: the heaviest, j = 0, first)
+    const int b = bhk / p.H_kv;
+    const int G = p.H / p.H_kv;   // query heads sharing this key/value head
+    const int bh_first = b * p.H + (bhk % p.H_kv) * G;
     const int L = seq_len(p, b, threadIdx.x == 0 && j == 0);
     const int k0 = j * C::BN;
 
     if (k0 >= L) {
         // Every key of this block is padding: dK = dV = 0 and no dQ contribution.
         const int rows = min(C::BN, p.N - k0);
-        uint4* dk = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.dk) + ((size_t)bh * p.N + k0) * D);
-        uint4* dv = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.dv) + ((size_t)bh * p.N + k0) * D);
+        uint4* dk = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.dk) + ((size_t)bhk * p.N + k0) * D);
+        uint4* dv = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.dv) + ((size_t)bhk * p.N + k0) * D);
         for (int i = threadIdx.x; i < rows * D / 8; i += blockDim.x) {
             dk[i] = make_uint4(0, 0, 0, 0);
             dv[i] = make_uint4(0, 0, 0, 0);
@@ -307,10 +316,16 @@ __global__ void __launch_bounds__(512, 1)
     // at query block j and wrap, so the key blocks of a head add into different query
     // blocks at any moment instead of all hammering the same accumulator lines.
     const int i_start = p.causal ? j : 0;
-    const int n_it = n_q - i_start;
+    // Step it visits query head q_head(it) of the group (each head in turn) and query block
+    // q_block(it) of that head; dK and dV accumulate over every step, so they sum over the
+    // group's query heads.
+    const int n_it_head = n_q - i_start;
+    const int n_it = G * n_it_head;
+    auto q_head = [&](int it) { return bh_first + it / n_it_head; };
     auto q_block = [&](int it) {
-        if (p.causal) return j + it;
-        const int i = j + it;
+        const int r = it % n_it_head;
+        if (p.causal) return j + r;
+        const int i = j + r;
         return i < n_q ? i : i - n_q;
     };
 
@@ -349,7 +364,7 @@ __global__ void __launch_bounds__(512, 1)
         // ------------------------------------------------------------ dQ drain
         const int r = threadIdx.x - 384;                // TMEM lane
         const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
-        const float factor = head_bound_factor(p, bh);
+        const float factor = head_bound_factor(p, bhk);
         // Named barriers have no timeout: every drain thread executes each of them, also after
         // a failed wait (`ok` then only skips the work).
         bool ok = true;
@@ -360,7 +375,7 @@ __global__ void __launch_bounds__(512, 1)
             {
                 const int q = q0 + r;
                 s_scale[r] =
-                    q < p.N ? fixed_point_scale(p.dOnorm[(size_t)bh * p.N + q], factor) : 0.f;
+                    q < p.N ? fixed_point_scale(p.dOnorm[(size_t)q_head(it) * p.N + q], factor) : 0.f;
             }
             named_barrier(2, 128);
             const float* sc = s_scale;
@@ -376,7 +391,7 @@ __global__ void __launch_bounds__(512, 1)
                 for (int q = 0; q < NV / 32; ++q) reg_fence32(v + 32 * q);
                 tc_fence_before();
                 mbar_arrive(bar_dqempty);           // B may take the next dP^T
-                int* acc = p.dq_acc + ((size_t)bh * p.N_pad + q0) * D;
+                int* acc = p.dq_acc + ((size_t)q_head(it) * p.N_pad + q0) * D;
                 if constexpr (D == 128) {
                     // dQ^T: lane = feature r, column = query e; a warp instruction covers 32
                     // consecutive features of one query row: one 128-byte line.
@@ -416,8 +431,8 @@ __global__ void __launch_bounds__(512, 1)
         prefetch_tensormap(&tmDO);
         mbar_arrive_expect_tx(bar_kv, 2 * C::KV_TILE_BYTES);
         for (int c = 0; c < C::KCH; ++c) {
-            tma_load_3d(smem + C::SMEM_K + c * C::CHUNK_BYTES, &tmK, bar_kv, c * 64, k0, bh);
-            tma_load_3d(smem + C::SMEM_V + c * C::CHUNK_BYTES, &tmV, bar_kv, c * 64, k0, bh);
+            tma_load_3d(smem + C::SMEM_K + c * C::CHUNK_BYTES, &tmK, bar_kv, c * 64, k0, bhk);
+            tma_load_3d(smem + C::SMEM_V + c * C::CHUNK_BYTES, &tmV, bar_kv, c * 64, k0, bhk);
         }
         int it = 0;
         for (; it < n_it; ++it) {
@@ -428,9 +443,9 @@ __global__ void __launch_bounds__(512, 1)
             mbar_arrive_expect_tx(&bar_qfull[s], 2 * C::Q_TILE_BYTES);
             for (int c = 0; c < C::KCH; ++c) {
                 tma_load_3d(smem + C::SMEM_Q + s * C::Q_TILE_BYTES + c * C::CHUNK_BYTES, &tmQ,
-                            &bar_qfull[s], c * 64, q0, bh);
+                            &bar_qfull[s], c * 64, q0, q_head(it));
                 tma_load_3d(smem + C::SMEM_DO + s * C::Q_TILE_BYTES + c * C::CHUNK_BYTES,
-                            &tmDO, &bar_qfull[s], c * 64, q0, bh);
+                            &tmDO, &bar_qfull[s], c * 64, q0, q_head(it));
             }
         }
         // Do not leave while our copies may still be landing in shared memory.
@@ -556,8 +571,9 @@ __global__ void __launch_bounds__(512, 1)
         float staged = 0.f;
         auto load_vectors = [&](int it) {
             const int q = q_block(it) * C::BM + (ct & 127);
-            if (ct < 128) staged = q < p.N ? -p.lse[(size_t)bh * p.N + q] * kLog2e : -INFINITY;
-            else staged = q < p.N ? p.Dvec[(size_t)bh * p.N + q] : 0.f;
+            const size_t hrow = (size_t)q_head(it) * p.N;
+            if (ct < 128) staged = q < p.N ? -p.lse[hrow + q] * kLog2e : -INFINITY;
+            else staged = q < p.N ? p.Dvec[hrow + q] : 0.f;
         };
         auto store_vectors = [&](int it) {
             if (ct < 128) s_lse2[(it & 1) * C::BM + ct] = staged;
@@ -672,7 +688,7 @@ __global__ void __launch_bounds__(512, 1)
         if (__all_sync(0xffffffffu, ok)) {
             tc_fence_after();
             const bool in_range = kidx < p.N;
-            const size_t off = ((size_t)bh * p.N + (in_range ? kidx : 0)) * D;
+            const size_t off = ((size_t)bhk * p.N + (in_range ? kidx : 0)) * D;
             const uint32_t col0 = h ? C::TM_DK : C::TM_DV;
             const float mul = h ? p.scale : 1.0f;
             __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(h ? p.dk : p.dv) + off;
@@ -722,9 +738,10 @@ cudaError_t launch_bwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
     }
     const int BH = p.B * p.H;
     const int n_kv = (p.N + C::BN - 1) / C::BN;
+    const int BHkv = p.B * p.H_kv;
     const dim3 chunks(p.N_pad / 128, BH);
     fa_bwd_pre_kernel<D><<<chunks, 256, 0, stream>>>(p);
-    fa_bwd_kernel<D><<<BH * n_kv, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
+    fa_bwd_kernel<D><<<BHkv * n_kv, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
     fa_bwd_dq_kernel<D><<<chunks, 256, 0, stream>>>(p);
     return cudaGetLastError();
 }

@@ -116,6 +116,7 @@ extern "C" FA_API fa_status fa_bwd_noalloc(const void* q, const void* k, const v
     p.H = H;
     p.N = N;
     p.N_pad = Np;
+    p.H_kv = H;
     p.scale = scale;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;

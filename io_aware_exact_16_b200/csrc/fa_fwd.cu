@@ -87,6 +87,8 @@ __global__ void __launch_bounds__(384, 1)
     const int h = blockIdx.y;
     const int b = blockIdx.z;
     const int bh = b * p.H + h;
+    // Grouped-query attention: consecutive query heads share one key/value head.
+    const int bh_kv = b * p.H_kv + h / (p.H / p.H_kv);
     const int q_base = cta_x * C::ROWS_PER_CTA;
 
     int L = p.N;
@@ -170,12 +172,12 @@ __global__ void __launch_bounds__(384, 1)
                 mbar_arrive_expect_tx(&bar_kfull[s], C::KV_TILE_BYTES);
                 for (int c = 0; c < C::KCH; ++c)
                     tma_load_3d(smem + C::SMEM_K + s * C::KV_TILE_BYTES + c * C::CHUNK_BYTES, &tmK,
-                                &bar_kfull[s], c * 64, j * C::BN, bh);
+                                &bar_kfull[s], c * 64, j * C::BN, bh_kv);
                 if (!mbar_wait(&bar_vempty[s], ph ^ 1, p.timeout_ns, abort_flag)) { fail(); break; }
                 mbar_arrive_expect_tx(&bar_vfull[s], C::KV_TILE_BYTES);
                 for (int c = 0; c < C::KCH; ++c)
                     tma_load_3d(smem + C::SMEM_V + s * C::KV_TILE_BYTES + c * C::CHUNK_BYTES, &tmV,
-                                &bar_vfull[s], c * 64, j * C::BN, bh);
+                                &bar_vfull[s], c * 64, j * C::BN, bh_kv);
             }
             // Do not leave the CTA while our copies may still be landing in shared memory.
             for (int j = max(0, n - C::STAGES); j < n; ++j) {

@@ -19,6 +19,7 @@ struct FwdParams {
     const int* seqlens;    // device int32 [B] or nullptr
     int* err;              // device error flag
     int H, N;
+    int H_kv;              // key/value heads; query head h reads K/V head h / (H / H_kv)
     float scale_log2;      // scale * log2(e)
     int causal;
     uint64_t timeout_ns;
@@ -40,6 +41,7 @@ struct BwdParams {
     const int* seqlens;
     int* err;
     int B, H, N, N_pad;
+    int H_kv;              // key/value heads (H % H_kv == 0); dK, dV are [B, H_kv, N, d]
     float scale;
     float scale_log2;
     int causal;

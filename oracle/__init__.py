@@ -207,3 +207,46 @@ def attention_bwd(q, k, v, do, scale: float, causal: bool, seqlens=None):
             for n in out:
                 out[n][b, h] = r[n]
     return out
+
+
+def _kv_index(H: int, H_kv: int) -> list[int]:
+    """Key/value head of each query head: consecutive groups of H / H_kv query heads share one."""
+    if H_kv < 1 or H % H_kv != 0:
+        raise ValueError("H_kv must divide H")
+    G = H // H_kv
+    return [h // G for h in range(H)]
+
+
+def attention_fwd_gqa(q, k, v, scale: float, causal: bool, seqlens=None):
+    """Grouped-query attention: q [B, H, N, d], k, v [B, H_kv, N, d].  Query head h attends with
+    key/value head h // (H / H_kv) (multi-query attention when H_kv = 1; FlashAttention (DE),
+    FlashAttention-2 section).  Each head is the plain definition (``head_fwd``)."""
+    q, k, v = as_f64(q), as_f64(k), as_f64(v)
+    B, H, N, d = q.shape
+    kv = _kv_index(H, k.shape[1])
+    Ls = _lengths(seqlens, B, N)
+    O = np.empty((B, H, N, d), np.float64)
+    lse = np.empty((B, H, N), np.float64)
+    for b in range(B):
+        for h in range(H):
+            O[b, h], lse[b, h] = head_fwd(q[b, h], k[b, kv[h]], v[b, kv[h]], scale, causal, Ls[b])
+    return O, lse
+
+
+def attention_bwd_gqa(q, k, v, do, scale: float, causal: bool, seqlens=None):
+    """Backward of ``attention_fwd_gqa``: dQ per query head; dK, dV of a key/value head are the
+    sums over the query heads that read it (each summand from ``head_bwd``)."""
+    q, k, v, do = as_f64(q), as_f64(k), as_f64(v), as_f64(do)
+    B, H, N, d = q.shape
+    H_kv = k.shape[1]
+    kv = _kv_index(H, H_kv)
+    Ls = _lengths(seqlens, B, N)
+    out = {"dq": np.empty((B, H, N, d)), "o": np.empty((B, H, N, d)), "lse": np.empty((B, H, N)),
+           "dk": np.zeros((B, H_kv, N, d)), "dv": np.zeros((B, H_kv, N, d))}
+    for b in range(B):
+        for h in range(H):
+            r = head_bwd(q[b, h], k[b, kv[h]], v[b, kv[h]], do[b, h], scale, causal, Ls[b])
+            out["dq"][b, h], out["o"][b, h], out["lse"][b, h] = r["dq"], r["o"], r["lse"]
+            out["dk"][b, kv[h]] += r["dk"]
+            out["dv"][b, kv[h]] += r["dv"]
+    return out

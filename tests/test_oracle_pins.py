@@ -358,3 +358,41 @@ def test_pins_catch_planted_slips(kind):
     O, dq, dk, dv = torch_reference(q, k, v, do, 0.3, causal, N)
     worst = max(np.abs(got[n] - r).max() for n, r in (("o", O), ("dq", dq), ("dk", dk), ("dv", dv)))
     assert worst > 1e-6
+
+
+# ---------------------------------------------------------------- grouped-query attention
+def test_gqa_with_one_query_head_per_kv_head_is_plain_attention():
+    g = torch.Generator().manual_seed(50)
+    q, k, v, do = ((torch.randn((2, 3, 20, 8), generator=g)).to(torch.bfloat16) for _ in range(4))
+    a = oracle.attention_bwd_gqa(q, k, v, do, 0.3, True, [20, 11])
+    b = oracle.attention_bwd(q, k, v, do, 0.3, True, [20, 11])
+    for n in ("o", "lse", "dq", "dk", "dv"):
+        np.testing.assert_array_equal(a[n], b[n])
+
+
+@pytest.mark.parametrize("H,H_kv,causal", [(4, 2, False), (3, 1, True)])
+def test_gqa_gradients_match_central_differences(H, H_kv, causal):
+    """A shared key/value element feeds several query heads: its gradient is their sum."""
+    N, d = 6, 4
+    g = torch.Generator().manual_seed(51 + H)
+    q = torch.randn((1, H, N, d), generator=g).to(torch.bfloat16).double().numpy()
+    k = torch.randn((1, H_kv, N, d), generator=g).to(torch.bfloat16).double().numpy()
+    v = torch.randn((1, H_kv, N, d), generator=g).to(torch.bfloat16).double().numpy()
+    do = torch.randn((1, H, N, d), generator=g).to(torch.bfloat16).double().numpy()
+    grads = oracle.attention_bwd_gqa(q, k, v, do, 0.6, causal)
+    h = 1e-6
+
+    def loss(q_, k_, v_):
+        O, _ = oracle.attention_fwd_gqa(q_, k_, v_, 0.6, causal)
+        return float((O * do).sum())
+
+    for name, arr, grad in (("q", q, grads["dq"]), ("k", k, grads["dk"]), ("v", v, grads["dv"])):
+        fd = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            args = {"q": q.copy(), "k": k.copy(), "v": v.copy()}
+            args[name][idx] += h
+            lp = loss(args["q"], args["k"], args["v"])
+            args[name][idx] -= 2 * h
+            lm = loss(args["q"], args["k"], args["v"])
+            fd[idx] = (lp - lm) / (2 * h)
+        assert np.abs(fd - grad).max() <= 1e-6 * max(1.0, np.abs(grad).max()), name

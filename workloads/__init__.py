@@ -10,7 +10,8 @@ Input recipe (one generator per workload, ``torch.Generator().manual_seed(seed)`
 * key-padding lengths, when the workload has them, are drawn FIRST from the generator as
   ``L_b ~ UniformInt[lo, hi]`` inclusive, one per batch entry;
 * then Q, K, V and dO are drawn in that order as fp32 ``std * N(0, 1)`` of shape
-  ``[B, H, N, d]`` and rounded to bf16 (round to nearest even, torch ``.to(bfloat16)``).
+  ``[B, H, N, d]`` (K and V ``[B, H_kv, N, d]`` for grouped-query workloads) and rounded to
+  bf16 (round to nearest even, torch ``.to(bfloat16)``).
 
 The workload shapes follow the pages' own workloads: GPT-2 at sequence length 1K and
 BERT-large at 512 (FlashAttention (DE), "Empirische Ergebnisse"), the 8K-32K long-context
@@ -40,6 +41,12 @@ class Workload:
     # inclusive range of key-padding lengths, or None for "every key is valid"
     pad_range: Optional[tuple[int, int]] = None
     backward: bool = True
+    # key/value heads (grouped-query attention); None means H (one K/V head per query head)
+    H_kv: Optional[int] = None
+
+    @property
+    def kv_heads(self) -> int:
+        return self.H if self.H_kv is None else self.H_kv
 
     @property
     def scale(self) -> float:
@@ -88,8 +95,9 @@ def all_sweep() -> list[Workload]:
 
 
 def custom(B: int, H: int, N: int, d: int, causal: bool, seed: int, std: float = 1.0,
-           pad_range: Optional[tuple[int, int]] = None, name: str = "custom") -> Workload:
-    return Workload(name, B, H, N, d, causal, seed, std, pad_range)
+           pad_range: Optional[tuple[int, int]] = None, name: str = "custom",
+           H_kv: Optional[int] = None) -> Workload:
+    return Workload(name, B, H, N, d, causal, seed, std, pad_range, H_kv=H_kv)
 
 
 @dataclasses.dataclass
@@ -109,17 +117,18 @@ def make_inputs(w: Workload, with_grad: bool = True) -> Inputs:
         lo, hi = w.pad_range
         seqlens = torch.randint(lo, hi + 1, (w.B,), generator=g, dtype=torch.int64).to(torch.int32)
     shape = (w.B, w.H, w.N, w.d)
+    kv_shape = (w.B, w.kv_heads, w.N, w.d)
 
-    def draw() -> torch.Tensor:
-        x = torch.randn(shape, generator=g, dtype=torch.float32)
+    def draw(sh) -> torch.Tensor:
+        x = torch.randn(sh, generator=g, dtype=torch.float32)
         if w.std != 1.0:
             x.mul_(w.std)
         return x.to(torch.bfloat16)
 
-    q = draw()
-    k = draw()
-    v = draw()
-    do = draw() if with_grad else torch.empty(0, dtype=torch.bfloat16)
+    q = draw(shape)
+    k = draw(kv_shape)
+    v = draw(kv_shape)
+    do = draw(shape) if with_grad else torch.empty(0, dtype=torch.bfloat16)
     return Inputs(q, k, v, do, seqlens)
 
 
