@@ -144,6 +144,37 @@ FA_API fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const v
                             fa_stream_t stream);
 
 /*
+ * Packed variable-length sequences.  The pages print no packed layout; they speak of batches
+ * whose sequences differ in length (the padded BERT workload of FlashAttention (DE),
+ * "Empirische Ergebnisse").  This is the same computation with the sequences stored back to
+ * back instead of padded to a common length, so that no padding row is read or written.
+ * Sequence b is rows [cu_seqlens[b], cu_seqlens[b+1]) of
+ *   q, o, dO, dq   bf16 [total, H, d]      (row t, head h at (t * H + h) * d)
+ *   k, v, dk, dv   bf16 [total, H_kv, d]
+ *   lse            fp32 [H, total]          (natural-log units, as in fa_fwd)
+ * and is an independent attention problem: its queries attend to its own keys only (and, when
+ * causal, to keys j <= i of the same sequence, counted from the sequence's first row).  H_kv
+ * follows fa_fwd_gqa.  Rows of `o`, `lse`, `dq`, `dk`, `dv` outside every sequence
+ * ([cu_seqlens[B], total)) are not written.
+ *   cu_seqlens   device int32 [B + 1], 4-byte aligned, non-decreasing, cu_seqlens[0] >= 0,
+ *                cu_seqlens[B] <= total; empty sequences are allowed.
+ *   max_seqlen   >= the longest sequence (it sizes the grid and the backward workspace:
+ *                fa_bwd_workspace_size(B, H, max_seqlen, d)).
+ * A sequence that breaks these rules (found on the device) is skipped and FA_ERR_INVALID_ARG
+ * is recorded for fa_check_device_error.  Host-side checks as in fa_fwd, plus total >= 1 and
+ * total * H * d < 2^31.  The padded accumulators of the backward workspace keep the
+ * [B, H, max_seqlen] shape.
+ */
+FA_API fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                               const int* cu_seqlens, int B, int max_seqlen, int total, int H,
+                               int H_kv, int d, float scale, int causal, fa_stream_t stream);
+FA_API fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
+                               const void* dO, const float* lse, void* dq, void* dk, void* dv,
+                               const int* cu_seqlens, int B, int max_seqlen, int total, int H,
+                               int H_kv, int d, float scale, int causal, void* workspace,
+                               size_t workspace_bytes, fa_stream_t stream);
+
+/*
  * fa_bwd_noalloc -- the backward pass without any device allocation.  The pages have no
  * counterpart of this entry point; it exists for callers that cannot allocate device memory:
  * a process that reserves its whole device-memory budget for its own pool up front, or a

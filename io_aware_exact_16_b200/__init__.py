@@ -39,6 +39,12 @@ _lib.fa_fwd_gqa.restype = _i
 _lib.fa_bwd_gqa.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                             ctypes.c_float, _i, _vp, _vp, ctypes.c_size_t, _vp]
 _lib.fa_bwd_gqa.restype = _i
+_lib.fa_fwd_varlen.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                               ctypes.c_float, _i, _vp]
+_lib.fa_fwd_varlen.restype = _i
+_lib.fa_bwd_varlen.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                               _i, _i, ctypes.c_float, _i, _vp, ctypes.c_size_t, _vp]
+_lib.fa_bwd_varlen.restype = _i
 _lib.fa_bwd_workspace_size.argtypes = [_i, _i, _i, _i]
 _lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
 _lib.fa_check_device_error.argtypes = [_vp]
@@ -49,7 +55,8 @@ _lib.fa_status_string.argtypes = [_i]
 _lib.fa_status_string.restype = ctypes.c_char_p
 
 # Every symbol include/fa.h declares.
-EXPORTED = ("fa_fwd", "fa_bwd", "fa_fwd_gqa", "fa_bwd_gqa", "fa_bwd_workspace_size",
+EXPORTED = ("fa_fwd", "fa_bwd", "fa_fwd_gqa", "fa_bwd_gqa", "fa_fwd_varlen", "fa_bwd_varlen",
+            "fa_bwd_workspace_size",
             "fa_check_device_error", "fa_set_wait_timeout_ns", "fa_status_string",
             "fa_bwd_noalloc")
 
@@ -167,6 +174,81 @@ def backward(q, k, v, o, do, lse, causal: bool = False, seqlens: Optional[torch.
                          _stream_handle(dev))
     if st != FA_OK:
         raise FAError(st, "fa_bwd_gqa")
+    return dq, dk, dv
+
+
+def _check_packed(q, k, cu_seqlens, max_seqlen):
+    """Shapes of the packed layout: q [T, H, d], k [T, H_kv, d], cu_seqlens int32 [B + 1]."""
+    if q.dim() != 3 or k.dim() != 3:
+        raise ValueError("packed q, k, v must be [total, heads, d]")
+    T, H, d = q.shape
+    H_kv = k.shape[1]
+    if H_kv < 1 or H % H_kv != 0:
+        raise ValueError(f"key/value heads {H_kv} must divide query heads {H}")
+    if (cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2
+            or cu_seqlens.device != q.device or not cu_seqlens.is_contiguous()):
+        raise ValueError("cu_seqlens must be a contiguous int32 tensor [B + 1] on q's device")
+    if int(max_seqlen) < 1:
+        raise ValueError("max_seqlen must be >= 1")
+    return T, H, H_kv, d, cu_seqlens.numel() - 1
+
+
+def forward_varlen(q, k, v, cu_seqlens, max_seqlen: int, causal: bool = False,
+                   scale: Optional[float] = None, out=None, lse=None):
+    """``fa_fwd_varlen``: packed sequences, q [T, H, d], k and v [T, H_kv, d]; sequence b is
+    rows cu_seqlens[b] .. cu_seqlens[b+1].  Returns (O bf16 [T, H, d], lse fp32 [H, T])."""
+    T, H, H_kv, d, B = _check_packed(q, k, cu_seqlens, max_seqlen)
+    dev = q.device
+    _check_qkv("q", q, (T, H, d), dev)
+    for name, t in (("k", k), ("v", v)):
+        _check_qkv(name, t, (T, H_kv, d), dev)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check_qkv("out", out, (T, H, d), dev)
+    if lse is None:
+        lse = torch.empty((H, T), dtype=torch.float32, device=dev)
+    elif lse.dtype != torch.float32 or tuple(lse.shape) != (H, T) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 tensor [H, T]")
+    sc = float(scale) if scale is not None else 1.0 / (d ** 0.5)
+    st = _lib.fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                            lse.data_ptr(), cu_seqlens.data_ptr(), B, int(max_seqlen), T, H,
+                            H_kv, d, sc, int(bool(causal)), _stream_handle(dev))
+    if st != FA_OK:
+        raise FAError(st, "fa_fwd_varlen")
+    return out, lse
+
+
+def backward_varlen(q, k, v, o, do, lse, cu_seqlens, max_seqlen: int, causal: bool = False,
+                    scale: Optional[float] = None, dq=None, dk=None, dv=None,
+                    workspace: Optional[torch.Tensor] = None):
+    """``fa_bwd_varlen``: gradients of ``forward_varlen``; returns (dQ, dK, dV) in bf16 shaped
+    like q, k and v."""
+    T, H, H_kv, d, B = _check_packed(q, k, cu_seqlens, max_seqlen)
+    dev = q.device
+    for name, t in (("q", q), ("o", o), ("do", do)):
+        _check_qkv(name, t, (T, H, d), dev)
+    for name, t in (("k", k), ("v", v)):
+        _check_qkv(name, t, (T, H_kv, d), dev)
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (H, T) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 tensor [H, T]")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check_qkv("dq", dq, (T, H, d), dev)
+    for name, t in (("dk", dk), ("dv", dv)):
+        _check_qkv(name, t, (T, H_kv, d), dev)
+    need = bwd_workspace_size(B, H, int(max_seqlen), d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    sc = float(scale) if scale is not None else 1.0 / (d ** 0.5)
+    st = _lib.fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                            lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                            cu_seqlens.data_ptr(), B, int(max_seqlen), T, H, H_kv, d, sc,
+                            int(bool(causal)), workspace.data_ptr(),
+                            workspace.numel() * workspace.element_size(), _stream_handle(dev))
+    if st != FA_OK:
+        raise FAError(st, "fa_bwd_varlen")
     return dq, dk, dv
 
 

@@ -110,6 +110,75 @@ bool make_bf16_map(CUtensorMap* map, const void* base, int d, int N, int BH, int
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_bf16_map_packed(CUtensorMap* map, const void* base, int d, int Hx, int T, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)Hx, (cuuint64_t)T};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)Hx * d * 2};
+    cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+namespace {
+
+// Tensor map of a user tensor with Hx heads: head-major [B, Hx, N, d] or packed [T, Hx, d].
+bool user_map(CUtensorMap* map, const void* base, int d, int B, int Hx, int N, int T,
+              bool packed) {
+    return packed ? make_bf16_map_packed(map, base, d, Hx, T, 128)
+                  : make_bf16_map(map, base, d, N, B * Hx, 128);
+}
+
+// Checks shared by the head-major and packed entry points; T = 0 for head-major.
+fa_status check_layout(int B, int H, int H_kv, int N, int d, float scale, const int* seqlens,
+                       const int* cu_seqlens, int T) {
+    fa_status st = check_common(B, H, N, d, scale);
+    if (st != FA_OK) return st;
+    if (H_kv < 1 || H_kv > H || H % H_kv != 0) return FA_ERR_INVALID_ARG;
+    if (seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u)) return FA_ERR_INVALID_ARG;
+    if (cu_seqlens) {
+        if (seqlens || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return FA_ERR_INVALID_ARG;
+        if (T < 1 || (long long)T * H * d >= (1ll << 31)) return FA_ERR_INVALID_ARG;
+    }
+    return FA_OK;
+}
+
+fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                   int H_kv, int N, int d, float scale, int causal, const int* seqlens,
+                   const int* cu_seqlens, int T, cudaStream_t stream) {
+    fa_status st = check_layout(B, H, H_kv, N, d, scale, seqlens, cu_seqlens, T);
+    if (st != FA_OK) return st;
+    if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return FA_ERR_INVALID_ARG;
+    DeviceState* dev = current_device(&st);
+    if (!dev) return st;
+
+    const bool packed = cu_seqlens != nullptr;
+    CUtensorMap tq, tk, tv;
+    if (!user_map(&tq, q, d, B, H, N, T, packed) || !user_map(&tk, k, d, B, H_kv, N, T, packed) ||
+        !user_map(&tv, v, d, B, H_kv, N, T, packed))
+        return FA_ERR_CUDA;
+    FwdParams p{};
+    p.o = o;
+    p.lse = lse;
+    p.seqlens = seqlens;
+    p.cu_seqlens = cu_seqlens;
+    p.T = T;
+    p.err = dev->err_flag;
+    p.H = H;
+    p.N = N;
+    p.H_kv = H_kv;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.causal = causal ? 1 : 0;
+    p.timeout_ns = g_timeout_ns.load();
+    if (launch_fwd(d, tq, tk, tv, p, B, dev->num_sms, stream) != cudaSuccess) return FA_ERR_CUDA;
+    return FA_OK;
+}
+
+}  // namespace
 }  // namespace fa
 
 using namespace fa;
@@ -135,35 +204,16 @@ void fa_set_wait_timeout_ns(uint64_t ns) {
 fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                      int H, int H_kv, int N, int d, float scale, int causal, const int* seqlens,
                      fa_stream_t stream) {
-    fa_status st = check_common(B, H, N, d, scale);
-    if (st != FA_OK) return st;
-    if (H_kv < 1 || H_kv > H || H % H_kv != 0) return FA_ERR_INVALID_ARG;
-    if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
-        return FA_ERR_INVALID_ARG;
-    if (seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u)) return FA_ERR_INVALID_ARG;
-    DeviceState* dev = current_device(&st);
-    if (!dev) return st;
+    return fwd_impl(q, k, v, o, lse, B, H, H_kv, N, d, scale, causal, seqlens, nullptr, 0,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
 
-    CUtensorMap tq, tk, tv;
-    if (!make_bf16_map(&tq, q, d, N, B * H, 128) || !make_bf16_map(&tk, k, d, N, B * H_kv, 128) ||
-        !make_bf16_map(&tv, v, d, N, B * H_kv, 128))
-        return FA_ERR_CUDA;
-    FwdParams p{};
-    p.o = o;
-    p.lse = lse;
-    p.seqlens = seqlens;
-    p.err = dev->err_flag;
-    p.H = H;
-    p.N = N;
-    p.H_kv = H_kv;
-    p.scale_log2 = scale * 1.4426950408889634f;
-    p.causal = causal ? 1 : 0;
-    p.timeout_ns = g_timeout_ns.load();
-    if (launch_fwd(d, tq, tk, tv, p, B, dev->num_sms, reinterpret_cast<cudaStream_t>(stream)) !=
-        cudaSuccess)
-        return FA_ERR_CUDA;
-    return FA_OK;
+fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                        const int* cu_seqlens, int B, int max_seqlen, int total, int H, int H_kv,
+                        int d, float scale, int causal, fa_stream_t stream) {
+    if (!cu_seqlens) return FA_ERR_INVALID_ARG;
+    return fwd_impl(q, k, v, o, lse, B, H, H_kv, max_seqlen, d, scale, causal, nullptr,
+                    cu_seqlens, total, reinterpret_cast<cudaStream_t>(stream));
 }
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
@@ -184,18 +234,17 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
     return bytes;
 }
 
-fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
-                     const void* dO, const float* lse, void* dq, void* dk, void* dv, int B, int H,
-                     int H_kv, int N, int d, float scale, int causal, const int* seqlens,
-                     void* workspace, size_t workspace_bytes, fa_stream_t stream) {
-    fa_status st = check_common(B, H, N, d, scale);
+static fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o,
+                          const void* dO, const float* lse, void* dq, void* dk, void* dv, int B,
+                          int H, int H_kv, int N, int d, float scale, int causal,
+                          const int* seqlens, const int* cu_seqlens, int T, void* workspace,
+                          size_t workspace_bytes, cudaStream_t stream) {
+    fa_status st = check_layout(B, H, H_kv, N, d, scale, seqlens, cu_seqlens, T);
     if (st != FA_OK) return st;
-    if (H_kv < 1 || H_kv > H || H % H_kv != 0) return FA_ERR_INVALID_ARG;
     if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dO) ||
         !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
         return FA_ERR_INVALID_ARG;
-    if (seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u)) return FA_ERR_INVALID_ARG;
     if (!workspace || !aligned16(workspace) || workspace_bytes < fa_bwd_workspace_size(B, H, N, d))
         return FA_ERR_WORKSPACE;
     DeviceState* dev = current_device(&st);
@@ -224,6 +273,8 @@ fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
     p.headmax = static_cast<float*>(take((size_t)BH * (Np / 128) * 2 * sizeof(float)));
     p.dq_acc = static_cast<int*>(take((size_t)BH * Np * d * sizeof(int)));
     p.seqlens = seqlens;
+    p.cu_seqlens = cu_seqlens;
+    p.T = T;
     p.err = dev->err_flag;
     p.B = B;
     p.H = H;
@@ -235,13 +286,32 @@ fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
     p.causal = causal ? 1 : 0;
     p.timeout_ns = g_timeout_ns.load();
 
+    const bool packed = cu_seqlens != nullptr;
     CUtensorMap tq, tk, tv, tdo;
-    if (!make_bf16_map(&tq, q, d, N, BH, 128) || !make_bf16_map(&tk, k, d, N, B * H_kv, 128) ||
-        !make_bf16_map(&tv, v, d, N, B * H_kv, 128) || !make_bf16_map(&tdo, dO, d, N, BH, 128))
+    if (!user_map(&tq, q, d, B, H, N, T, packed) || !user_map(&tk, k, d, B, H_kv, N, T, packed) ||
+        !user_map(&tv, v, d, B, H_kv, N, T, packed) || !user_map(&tdo, dO, d, B, H, N, T, packed))
         return FA_ERR_CUDA;
-    if (launch_bwd(d, tq, tk, tv, tdo, p, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-        return FA_ERR_CUDA;
+    if (launch_bwd(d, tq, tk, tv, tdo, p, stream) != cudaSuccess) return FA_ERR_CUDA;
     return FA_OK;
+}
+
+fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
+                     const void* dO, const float* lse, void* dq, void* dk, void* dv, int B, int H,
+                     int H_kv, int N, int d, float scale, int causal, const int* seqlens,
+                     void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+    return bwd_impl(q, k, v, o, dO, lse, dq, dk, dv, B, H, H_kv, N, d, scale, causal, seqlens,
+                    nullptr, 0, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
+                        const void* dO, const float* lse, void* dq, void* dk, void* dv,
+                        const int* cu_seqlens, int B, int max_seqlen, int total, int H, int H_kv,
+                        int d, float scale, int causal, void* workspace, size_t workspace_bytes,
+                        fa_stream_t stream) {
+    if (!cu_seqlens) return FA_ERR_INVALID_ARG;
+    return bwd_impl(q, k, v, o, dO, lse, dq, dk, dv, B, H, H_kv, max_seqlen, d, scale, causal,
+                    nullptr, cu_seqlens, total, workspace, workspace_bytes,
+                    reinterpret_cast<cudaStream_t>(stream));
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,

@@ -102,18 +102,6 @@ __device__ __forceinline__ void record_error(int* err, int code) {
     if (err) atomicCAS(err, 0, code);
 }
 
-__device__ __forceinline__ int seq_len(const BwdParams& p, int b, bool report) {
-    int L = p.N;
-    if (p.seqlens != nullptr) {
-        L = p.seqlens[b];
-        if (L < 1 || L > p.N) {
-            if (report) record_error(p.err, kErrInvalidArg);
-            L = L < 1 ? 1 : p.N;
-        }
-    }
-    return L;
-}
-
 // Head constant 2 max_j |v_j| max_{j,l} |k_jl| from the per-chunk maxima (same arithmetic in
 // every kernel that needs it, so every kernel derives the same scales).
 __device__ __forceinline__ float head_bound_factor(const BwdParams& p, int bh) {
@@ -157,14 +145,18 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p) {
     const int part = threadIdx.x % TPR;
     // Blocks of the first B * H_kv heads also scan key/value head bh for the bound maxima; only
     // keys some query can see enter them (padded keys contribute nothing to dQ).
+    const bool packed = p.cu_seqlens != nullptr;
     const bool kv_head = bh < p.B * p.H_kv;
-    const int L = kv_head ? seq_len(p, bh / p.H_kv, false) : 0;
+    const int bq = bh / p.H, bk = bh / p.H_kv;
+    const SeqExtent eq = sequence_extent(p, bq, false, packed);
+    const SeqExtent ek = kv_head ? sequence_extent(p, bk, false, packed) : SeqExtent{0, 0, 0};
+    const int L = ek.L;
     float vmax = 0.f, kmax = 0.f;
     for (int rr = threadIdx.x / TPR; rr < 128; rr += RPP) {
         const int n = chunk * 128 + rr;
         float dd = 0.f, nn = 0.f, vv = 0.f, ka = 0.f;
-        if (n < p.N) {
-            const size_t off = ((size_t)bh * p.N + n) * TPR + part;
+        if (n < eq.Lq) {
+            const size_t off = row_of(packed, bq, bh % p.H, p.H, p.N, eq.t0, n) * TPR + part;
             const uint4 a = reinterpret_cast<const uint4*>(p.dO)[off];
             const uint4 o = reinterpret_cast<const uint4*>(p.o)[off];
             const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
@@ -178,7 +170,7 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p) {
             }
         }
         if (n < L) {
-            const size_t off = ((size_t)bh * p.N + n) * TPR + part;
+            const size_t off = row_of(packed, bk, bh % p.H_kv, p.H_kv, p.N, ek.t0, n) * TPR + part;
             const uint4 v = reinterpret_cast<const uint4*>(p.v)[off];
             const uint4 k = reinterpret_cast<const uint4*>(p.k)[off];
             const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&v);
@@ -242,11 +234,14 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const BwdParams p) {
         s_factor = head_bound_factor(p, (bh / p.H) * p.H_kv + (bh % p.H) / (p.H / p.H_kv));
     __syncthreads();
     const float factor = s_factor;
+    const bool packed = p.cu_seqlens != nullptr;
+    const int b = bh / p.H;
+    const SeqExtent e = sequence_extent(p, b, false, packed);
     constexpr int PER_ROW = D / 8;  // 8 elements per thread-step
     for (int i = threadIdx.x; i < 128 * PER_ROW; i += 256) {
         const int rr = i / PER_ROW, c8 = (i % PER_ROW) * 8;
         const int n = chunk * 128 + rr;
-        if (n >= p.N) continue;
+        if (n >= e.Lq) continue;
         const float s = fixed_point_scale(p.dOnorm[(size_t)bh * p.N + n], factor);
         const float mul = s > 0.f ? p.scale / s : 0.f;  // 1 / s is a power of two: exact
         const int4* src = reinterpret_cast<const int4*>(p.dq_acc + ((size_t)bh * p.N_pad + n) * D + c8);
@@ -256,12 +251,13 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const BwdParams p) {
         out.y = pack_bf16x2((float)x.z * mul, (float)x.w * mul);
         out.z = pack_bf16x2((float)y.x * mul, (float)y.y * mul);
         out.w = pack_bf16x2((float)y.z * mul, (float)y.w * mul);
-        *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.dq) + ((size_t)bh * p.N + n) * D + c8) = out;
+        *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.dq) +
+                                  row_of(packed, b, bh % p.H, p.H, p.N, e.t0, n) * D + c8) = out;
     }
 }
 
 // ---------------------------------------------------------------------------- main kernel
-template <int D>
+template <int D, bool PACKED>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -271,8 +267,7 @@ __global__ void __launch_bounds__(512, 1)
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    const int n_q = (p.N + C::BM - 1) / C::BM;  // query blocks per head
-    const int n_kv = (p.N + C::BN - 1) / C::BN;
+    const int n_kv = (p.N + C::BN - 1) / C::BN;  // key blocks per head (of the longest sequence)
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_BAR);
     uint64_t* bar_kv = bars;
@@ -298,10 +293,21 @@ __global__ void __launch_bounds__(512, 1)
     const int b = bhk / p.H_kv;
     const int G = p.H / p.H_kv;   // query heads sharing this key/value head
     const int bh_first = b * p.H + (bhk % p.H_kv) * G;
-    const int L = seq_len(p, b, threadIdx.x == 0 && j == 0);
+    constexpr bool packed = PACKED;
+    const SeqExtent ext =
+        sequence_extent(p, b, threadIdx.x == 0 && j == 0 && bhk % p.H_kv == 0, packed);
+    const int L = ext.L;
+    const int n_q = (ext.Lq + C::BM - 1) / C::BM;  // query blocks of this sequence
     const int k0 = j * C::BN;
+    // TMA coordinates (y, z) of row n of query head qh (= b*H + h) and of this key/value head.
+    auto q_y = [&](int qh, int n) { return packed ? qh - b * p.H : n; };
+    auto q_z = [&](int qh, int n) { return packed ? ext.t0 + n : qh; };
+    const int kv_y = packed ? bhk % p.H_kv : k0;
+    const int kv_z = packed ? ext.t0 + k0 : bhk;
 
     if (k0 >= L) {
+        // Packed: these rows belong to no key of this sequence; nothing to write.
+        if (packed) return;
         // Every key of this block is padding: dK = dV = 0 and no dQ contribution.
         const int rows = min(C::BN, p.N - k0);
         uint4* dk = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.dk) + ((size_t)bhk * p.N + k0) * D);
@@ -375,7 +381,7 @@ __global__ void __launch_bounds__(512, 1)
             {
                 const int q = q0 + r;
                 s_scale[r] =
-                    q < p.N ? fixed_point_scale(p.dOnorm[(size_t)q_head(it) * p.N + q], factor) : 0.f;
+                    q < ext.Lq ? fixed_point_scale(p.dOnorm[(size_t)q_head(it) * p.N + q], factor) : 0.f;
             }
             named_barrier(2, 128);
             const float* sc = s_scale;
@@ -431,21 +437,22 @@ __global__ void __launch_bounds__(512, 1)
         prefetch_tensormap(&tmDO);
         mbar_arrive_expect_tx(bar_kv, 2 * C::KV_TILE_BYTES);
         for (int c = 0; c < C::KCH; ++c) {
-            tma_load_3d(smem + C::SMEM_K + c * C::CHUNK_BYTES, &tmK, bar_kv, c * 64, k0, bhk);
-            tma_load_3d(smem + C::SMEM_V + c * C::CHUNK_BYTES, &tmV, bar_kv, c * 64, k0, bhk);
+            tma_load_3d(smem + C::SMEM_K + c * C::CHUNK_BYTES, &tmK, bar_kv, c * 64, kv_y, kv_z);
+            tma_load_3d(smem + C::SMEM_V + c * C::CHUNK_BYTES, &tmV, bar_kv, c * 64, kv_y, kv_z);
         }
         int it = 0;
         for (; it < n_it; ++it) {
             const int s = it % C::QST;
             const uint32_t ph = (it / C::QST) & 1;
             const int q0 = q_block(it) * C::BM;
+            const int qh = q_head(it);
             if (!mbar_wait(&bar_qempty[s], ph ^ 1, p.timeout_ns, abort_flag)) { fail(); break; }
             mbar_arrive_expect_tx(&bar_qfull[s], 2 * C::Q_TILE_BYTES);
             for (int c = 0; c < C::KCH; ++c) {
                 tma_load_3d(smem + C::SMEM_Q + s * C::Q_TILE_BYTES + c * C::CHUNK_BYTES, &tmQ,
-                            &bar_qfull[s], c * 64, q0, q_head(it));
+                            &bar_qfull[s], c * 64, q_y(qh, q0), q_z(qh, q0));
                 tma_load_3d(smem + C::SMEM_DO + s * C::Q_TILE_BYTES + c * C::CHUNK_BYTES,
-                            &tmDO, &bar_qfull[s], c * 64, q0, q_head(it));
+                            &tmDO, &bar_qfull[s], c * 64, q_y(qh, q0), q_z(qh, q0));
             }
         }
         // Do not leave while our copies may still be landing in shared memory.
@@ -569,11 +576,16 @@ __global__ void __launch_bounds__(512, 1)
         // The global load is issued one iteration ahead (load_vectors) and stored to shared
         // memory at the end of the iteration (store_vectors), so its latency stays hidden.
         float staged = 0.f;
+        // lse of query head bh_first + g, position q: lse[lse_base + g * lse_hstride + q].
+        const size_t lse_hstride = packed ? (size_t)p.T : (size_t)p.N;
+        const size_t lse_base = lse_of(packed, b, bh_first - b * p.H, p.H, p.N, p.T, ext.t0, 0);
         auto load_vectors = [&](int it) {
             const int q = q_block(it) * C::BM + (ct & 127);
-            const size_t hrow = (size_t)q_head(it) * p.N;
-            if (ct < 128) staged = q < p.N ? -p.lse[hrow + q] * kLog2e : -INFINITY;
-            else staged = q < p.N ? p.Dvec[hrow + q] : 0.f;
+            const int g = it / n_it_head;  // head of the group
+            if (ct < 128)
+                staged = q < ext.Lq ? -p.lse[lse_base + (size_t)g * lse_hstride + q] * kLog2e
+                                    : -INFINITY;
+            else staged = q < ext.Lq ? p.Dvec[(size_t)(bh_first + g) * p.N + q] : 0.f;
         };
         auto store_vectors = [&](int it) {
             if (ct < 128) s_lse2[(it & 1) * C::BM + ct] = staged;
@@ -687,8 +699,9 @@ __global__ void __launch_bounds__(512, 1)
         if (ok) ok = mbar_wait(bar_done, 0, p.timeout_ns, abort_flag);  // every MMA finished
         if (__all_sync(0xffffffffu, ok)) {
             tc_fence_after();
-            const bool in_range = kidx < p.N;
-            const size_t off = ((size_t)bhk * p.N + (in_range ? kidx : 0)) * D;
+            const bool in_range = kidx < (packed ? L : p.N);
+            const size_t off =
+                row_of(packed, b, bhk % p.H_kv, p.H_kv, p.N, ext.t0, in_range ? kidx : 0) * D;
             const uint32_t col0 = h ? C::TM_DK : C::TM_DV;
             const float mul = h ? p.scale : 1.0f;
             __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(h ? p.dk : p.dv) + off;
@@ -724,13 +737,13 @@ __global__ void __launch_bounds__(512, 1)
     }
 }
 
-template <int D>
+template <int D, bool PACKED>
 cudaError_t launch_bwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream) {
     using C = BwdCfg<D>;
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(fa_bwd_kernel<D>,
+        cudaError_t e = cudaFuncSetAttribute(fa_bwd_kernel<D, PACKED>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
@@ -741,7 +754,7 @@ cudaError_t launch_bwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
     const int BHkv = p.B * p.H_kv;
     const dim3 chunks(p.N_pad / 128, BH);
     fa_bwd_pre_kernel<D><<<chunks, 256, 0, stream>>>(p);
-    fa_bwd_kernel<D><<<BHkv * n_kv, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
+    fa_bwd_kernel<D, PACKED><<<BHkv * n_kv, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
     fa_bwd_dq_kernel<D><<<chunks, 256, 0, stream>>>(p);
     return cudaGetLastError();
 }
@@ -750,8 +763,12 @@ cudaError_t launch_bwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 
 cudaError_t launch_bwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream) {
-    if (d == 64) return launch_bwd_d<64>(tq, tk, tv, tdo, p, stream);
-    return launch_bwd_d<128>(tq, tk, tv, tdo, p, stream);
+    const bool packed = p.cu_seqlens != nullptr;
+    if (d == 64)
+        return packed ? launch_bwd_d<64, true>(tq, tk, tv, tdo, p, stream)
+                      : launch_bwd_d<64, false>(tq, tk, tv, tdo, p, stream);
+    return packed ? launch_bwd_d<128, true>(tq, tk, tv, tdo, p, stream)
+                  : launch_bwd_d<128, false>(tq, tk, tv, tdo, p, stream);
 }
 
 }  // namespace fa

@@ -72,7 +72,7 @@ __device__ __forceinline__ void record_error(int* err, int code) {
     if (err) atomicCAS(err, 0, code);
 }
 
-template <int D>
+template <int D, bool PACKED>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -88,17 +88,19 @@ __global__ void __launch_bounds__(384, 1)
     const int b = blockIdx.z;
     const int bh = b * p.H + h;
     // Grouped-query attention: consecutive query heads share one key/value head.
-    const int bh_kv = b * p.H_kv + h / (p.H / p.H_kv);
+    const int h_kv = h / (p.H / p.H_kv);
     const int q_base = cta_x * C::ROWS_PER_CTA;
 
-    int L = p.N;
-    if (p.seqlens != nullptr) {
-        L = p.seqlens[b];
-        if (L < 1 || L > p.N) {
-            if (threadIdx.x == 0) record_error(p.err, kErrInvalidArg);
-            L = L < 1 ? 1 : p.N;
-        }
-    }
+    constexpr bool packed = PACKED;
+    const SeqExtent ext = sequence_extent(p, b, threadIdx.x == 0 && h == 0 && cta_x == 0, packed);
+    const int L = ext.L;
+    // Packed sequences shorter than the longest one leave whole CTAs without query rows.
+    if (q_base >= ext.Lq) return;
+    // TMA coordinates (y, z) of row n: head-major (n, b*H + h); packed (h, t0 + n).
+    auto q_y = [&](int n) { return packed ? h : n; };
+    auto q_z = [&](int n) { return packed ? ext.t0 + n : bh; };
+    auto kv_y = [&](int n) { return packed ? h_kv : n; };
+    auto kv_z = [&](int n) { return packed ? ext.t0 + n : b * p.H_kv + h_kv; };
     // Key blocks each query tile needs: keys j < lim, lim = min(L, last row + 1) if causal.
     auto blocks_for = [&](int row_end) {
         const int lim = p.causal ? min(L, row_end) : L;
@@ -163,7 +165,7 @@ __global__ void __launch_bounds__(384, 1)
             for (int t = 0; t < C::TILES; ++t)
                 for (int c = 0; c < C::KCH; ++c)
                     tma_load_3d(smem + C::SMEM_Q + t * C::Q_TILE_BYTES + c * C::CHUNK_BYTES, &tmQ,
-                                bar_q, c * 64, q_base + t * C::BM, bh);
+                                bar_q, c * 64, q_y(q_base + t * C::BM), q_z(q_base + t * C::BM));
             const int n = nblk1;
             for (int j = 0; j < n; ++j) {
                 const int s = j % C::STAGES;
@@ -172,12 +174,12 @@ __global__ void __launch_bounds__(384, 1)
                 mbar_arrive_expect_tx(&bar_kfull[s], C::KV_TILE_BYTES);
                 for (int c = 0; c < C::KCH; ++c)
                     tma_load_3d(smem + C::SMEM_K + s * C::KV_TILE_BYTES + c * C::CHUNK_BYTES, &tmK,
-                                &bar_kfull[s], c * 64, j * C::BN, bh_kv);
+                                &bar_kfull[s], c * 64, kv_y(j * C::BN), kv_z(j * C::BN));
                 if (!mbar_wait(&bar_vempty[s], ph ^ 1, p.timeout_ns, abort_flag)) { fail(); break; }
                 mbar_arrive_expect_tx(&bar_vfull[s], C::KV_TILE_BYTES);
                 for (int c = 0; c < C::KCH; ++c)
                     tma_load_3d(smem + C::SMEM_V + s * C::KV_TILE_BYTES + c * C::CHUNK_BYTES, &tmV,
-                                &bar_vfull[s], c * 64, j * C::BN, bh_kv);
+                                &bar_vfull[s], c * 64, kv_y(j * C::BN), kv_z(j * C::BN));
             }
             // Do not leave the CTA while our copies may still be landing in shared memory.
             for (int j = max(0, n - C::STAGES); j < n; ++j) {
@@ -383,9 +385,9 @@ __global__ void __launch_bounds__(384, 1)
         if (__all_sync(0xffffffffu, ok)) {
             tc_fence_after();
             const float inv_l = l > 0.f ? 1.0f / l : 0.f;
-            const bool in_range = row < p.N;
-            __nv_bfloat16* orow =
-                reinterpret_cast<__nv_bfloat16*>(p.o) + ((size_t)bh * p.N + (in_range ? row : 0)) * D;
+            const bool in_range = row < ext.Lq;
+            __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) +
+                                  row_of(packed, b, h, p.H, p.N, ext.t0, in_range ? row : 0) * D;
 #pragma unroll
             for (int q = 0; q < D / 32; ++q) {
                 uint32_t o[32];
@@ -406,7 +408,7 @@ __global__ void __launch_bounds__(384, 1)
             }
             if (in_range) {
                 // lse in natural-log units: (m + log2 l) * ln 2
-                p.lse[(size_t)bh * p.N + row] =
+                p.lse[lse_of(packed, b, h, p.H, p.N, p.T, ext.t0, row)] =
                     l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
             }
         } else {
@@ -423,20 +425,20 @@ __global__ void __launch_bounds__(384, 1)
     }
 }
 
-template <int D>
+template <int D, bool PACKED>
 cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const FwdParams& p, int B, cudaStream_t stream) {
     using C = FwdCfg<D>;
     static bool configured = false;  // attribute set once per process (idempotent if raced)
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(fa_fwd_kernel<D>,
+        cudaError_t e = cudaFuncSetAttribute(fa_fwd_kernel<D, PACKED>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         configured = true;
     }
     dim3 grid((p.N + C::ROWS_PER_CTA - 1) / C::ROWS_PER_CTA, p.H, B);
-    fa_fwd_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    fa_fwd_kernel<D, PACKED><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }
 
@@ -445,8 +447,12 @@ cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const FwdParams& p, int B, int num_sms, cudaStream_t stream) {
     (void)num_sms;
-    if (d == 64) return launch_fwd_d<64>(tq, tk, tv, p, B, stream);
-    return launch_fwd_d<128>(tq, tk, tv, p, B, stream);
+    const bool packed = p.cu_seqlens != nullptr;
+    if (d == 64)
+        return packed ? launch_fwd_d<64, true>(tq, tk, tv, p, B, stream)
+                      : launch_fwd_d<64, false>(tq, tk, tv, p, B, stream);
+    return packed ? launch_fwd_d<128, true>(tq, tk, tv, p, B, stream)
+                  : launch_fwd_d<128, false>(tq, tk, tv, p, B, stream);
 }
 
 }  // namespace fa

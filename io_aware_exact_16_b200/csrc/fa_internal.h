@@ -13,10 +13,16 @@ namespace fa {
 constexpr int kErrInvalidArg = FA_ERR_INVALID_ARG;
 constexpr int kErrTimeout = FA_ERR_TIMEOUT;
 
+// Two layouts of the user tensors.
+//   head-major: q, o, dO, dq [B, H, N, d]; k, v, dk, dv [B, H_kv, N, d]; lse [B, H, N].
+//   packed (cu_seqlens != nullptr): sequence b is rows [cu[b], cu[b+1]) of q, o, dO, dq
+//     [T, H, d] and of k, v, dk, dv [T, H_kv, d]; lse is [H, T]; N is the longest sequence.
 struct FwdParams {
-    void* o;               // bf16 [B, H, N, d]
-    float* lse;            // fp32 [B, H, N]
-    const int* seqlens;    // device int32 [B] or nullptr
+    void* o;               // bf16 [B, H, N, d] or packed [T, H, d]
+    float* lse;            // fp32 [B, H, N] or packed [H, T]
+    const int* seqlens;    // device int32 [B] key lengths (head-major only) or nullptr
+    const int* cu_seqlens; // device int32 [B + 1] packed sequence offsets or nullptr
+    int T;                 // packed: rows of the packed tensors
     int* err;              // device error flag
     int H, N;
     int H_kv;              // key/value heads; query head h reads K/V head h / (H / H_kv)
@@ -39,6 +45,8 @@ struct BwdParams {
     float* headmax;        // fp32 [B, H, N_pad/128, 2] workspace: per-chunk max |v_j|_2, max |k_jl|
     int* dq_acc;           // int32 [B, H, N_pad, d]    workspace: fixed-point dQ accumulator
     const int* seqlens;
+    const int* cu_seqlens; // packed layout (see FwdParams); the workspace stays [B, H, N_pad]
+    int T;
     int* err;
     int B, H, N, N_pad;
     int H_kv;              // key/value heads (H % H_kv == 0); dK, dV are [B, H_kv, N, d]
@@ -48,12 +56,66 @@ struct BwdParams {
     uint64_t timeout_ns;
 };
 
+#ifdef __CUDACC__
+// Where sequence b lives.  Head-major: rows [0, N) of its heads, keys valid below L (the key
+// length, N without seqlens).  Packed: rows [t0, t0 + L) and queries and keys both end at L;
+// offsets that do not describe rows inside [0, T) with L <= N are reported through the error
+// flag and the sequence is treated as empty (nothing read, nothing written).
+struct SeqExtent {
+    int t0;   // first packed row (0 head-major)
+    int L;    // valid keys
+    int Lq;   // query rows that exist (N head-major, L packed)
+};
+
+// `packed` must equal (p.cu_seqlens != nullptr); kernels compiled for one layout pass it as a
+// constant so that the other layout's state drops out.
+template <class P>
+__device__ __forceinline__ SeqExtent sequence_extent(const P& p, int b, bool report,
+                                                     bool packed) {
+    SeqExtent e{0, p.N, p.N};
+    if (packed) {
+        const int t0 = p.cu_seqlens[b], t1 = p.cu_seqlens[b + 1];
+        if (t0 < 0 || t1 < t0 || t1 - t0 > p.N || t1 > p.T) {
+            if (report) atomicCAS(p.err, 0, kErrInvalidArg);
+            e.t0 = 0;
+            e.L = e.Lq = 0;
+        } else {
+            e.t0 = t0;
+            e.L = e.Lq = t1 - t0;
+        }
+    } else if (p.seqlens != nullptr) {
+        int L = p.seqlens[b];
+        if (L < 1 || L > p.N) {
+            if (report) atomicCAS(p.err, 0, kErrInvalidArg);
+            L = L < 1 ? 1 : p.N;
+        }
+        e.L = L;
+    }
+    return e;
+}
+
+// Row (in units of d elements) of position n of head hx (of Hx heads) of sequence b.
+__device__ __forceinline__ size_t row_of(bool packed, int b, int hx, int Hx, int N, int t0,
+                                         int n) {
+    return packed ? (size_t)(t0 + n) * Hx + hx : ((size_t)b * Hx + hx) * N + n;
+}
+// Index of the lse entry of query position n of head h (of H heads) of sequence b.
+__device__ __forceinline__ size_t lse_of(bool packed, int b, int h, int H, int N, int T, int t0,
+                                         int n) {
+    return packed ? (size_t)h * T + t0 + n : ((size_t)b * H + h) * N + n;
+}
+#endif
+
 // Current bound on device-side waits (fa_set_wait_timeout_ns).
 uint64_t wait_timeout_ns();
 
 // Tensor maps: a bf16 [B*H, N, d] tensor seen as 3-D (d, N, B*H), 128-byte swizzle,
 // box = 64 columns x `box_rows` rows; rows past N read as zeros.
 bool make_bf16_map(CUtensorMap* map, const void* base, int d, int N, int BH, int box_rows);
+// A packed bf16 [T, Hx, d] tensor seen as 3-D (d, Hx, T), box = 64 columns x 1 head x
+// `box_rows` rows (the same 128-byte-swizzled shared tile); rows past T read as zeros.
+// Coordinates are (column, head, row).
+bool make_bf16_map_packed(CUtensorMap* map, const void* base, int d, int Hx, int T, int box_rows);
 
 cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const FwdParams& p, int B, int num_sms, cudaStream_t stream);

@@ -250,3 +250,54 @@ def attention_bwd_gqa(q, k, v, do, scale: float, causal: bool, seqlens=None):
             out["dk"][b, kv[h]] += r["dk"]
             out["dv"][b, kv[h]] += r["dv"]
     return out
+
+
+def _sequence_bounds(cu_seqlens, T: int) -> list[tuple[int, int]]:
+    """Rows [t0, t1) of each packed sequence; the offsets must be non-decreasing inside [0, T]."""
+    cu = [int(x) for x in np.asarray(as_f64(cu_seqlens)).ravel()]
+    if len(cu) < 2 or cu[0] < 0 or cu[-1] > T or any(a > b for a, b in zip(cu, cu[1:])):
+        raise ValueError("cu_seqlens must be non-decreasing offsets inside [0, T]")
+    return list(zip(cu[:-1], cu[1:]))
+
+
+def attention_fwd_varlen(q, k, v, cu_seqlens, scale: float, causal: bool):
+    """Packed sequences: q [T, H, d], k, v [T, H_kv, d]; sequence b is rows
+    cu_seqlens[b] .. cu_seqlens[b+1] and is its own attention problem of that length (causal
+    positions counted from its first row).  Returns (O [T, H, d], lse [H, T]); rows outside
+    every sequence stay 0 in O and NaN in lse."""
+    q, k, v = as_f64(q), as_f64(k), as_f64(v)
+    T, H, d = q.shape
+    kv = _kv_index(H, k.shape[1])
+    O = np.zeros((T, H, d), np.float64)
+    lse = np.full((H, T), np.nan, np.float64)
+    for t0, t1 in _sequence_bounds(cu_seqlens, T):
+        if t1 == t0:
+            continue
+        for h in range(H):
+            O[t0:t1, h], lse[h, t0:t1] = head_fwd(q[t0:t1, h], k[t0:t1, kv[h]], v[t0:t1, kv[h]],
+                                                  scale, causal)
+    return O, lse
+
+
+def attention_bwd_varlen(q, k, v, do, cu_seqlens, scale: float, causal: bool):
+    """Backward of ``attention_fwd_varlen``: per sequence and query head ``head_bwd``; dK, dV of
+    a key/value head summed over the query heads that read it.  Returns a dict with o, lse,
+    dq [T, H, d], dk, dv [T, H_kv, d] (rows outside every sequence: 0, lse NaN)."""
+    q, k, v, do = as_f64(q), as_f64(k), as_f64(v), as_f64(do)
+    T, H, d = q.shape
+    H_kv = k.shape[1]
+    kv = _kv_index(H, H_kv)
+    out = {"o": np.zeros((T, H, d)), "lse": np.full((H, T), np.nan), "dq": np.zeros((T, H, d)),
+           "dk": np.zeros((T, H_kv, d)), "dv": np.zeros((T, H_kv, d))}
+    for t0, t1 in _sequence_bounds(cu_seqlens, T):
+        if t1 == t0:
+            continue
+        for h in range(H):
+            r = head_bwd(q[t0:t1, h], k[t0:t1, kv[h]], v[t0:t1, kv[h]], do[t0:t1, h], scale,
+                         causal)
+            out["o"][t0:t1, h] = r["o"]
+            out["lse"][h, t0:t1] = r["lse"]
+            out["dq"][t0:t1, h] = r["dq"]
+            out["dk"][t0:t1, kv[h]] += r["dk"]
+            out["dv"][t0:t1, kv[h]] += r["dv"]
+    return out

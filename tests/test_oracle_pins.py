@@ -396,3 +396,85 @@ def test_gqa_gradients_match_central_differences(H, H_kv, causal):
             lm = loss(args["q"], args["k"], args["v"])
             fd[idx] = (lp - lm) / (2 * h)
         assert np.abs(fd - grad).max() <= 1e-6 * max(1.0, np.abs(grad).max()), name
+
+
+# ------------------------------------------------------------------ packed variable-length
+CU_PACK = [0, 3, 3, 8, 9, 13]   # lengths 3, 0 (empty), 5, 1, 4; rows 13..14 belong to no sequence
+
+
+def _packed(T, H, H_kv, d, seed):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn((T, H, d), generator=g).to(torch.bfloat16).double().numpy()
+    k = torch.randn((T, H_kv, d), generator=g).to(torch.bfloat16).double().numpy()
+    v = torch.randn((T, H_kv, d), generator=g).to(torch.bfloat16).double().numpy()
+    do = torch.randn((T, H, d), generator=g).to(torch.bfloat16).double().numpy()
+    return q, k, v, do
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_zero_query_gives_each_sequences_own_running_mean(causal):
+    """Q = 0: row i of a sequence averages the value rows of ITS sequence that it sees (all of
+    them, or its first i + 1 when causal), and lse = ln(count) exactly.  A slice boundary off
+    by one, or a sequence leaking into the next, changes the mean."""
+    T, H, H_kv, d = 15, 4, 2, 3
+    _, k, v, _ = _packed(T, H, H_kv, d, 61)
+    q = np.zeros((T, H, d))
+    O, lse = oracle.attention_fwd_varlen(q, k, v, np.array(CU_PACK), 0.7, causal)
+    for t0, t1 in zip(CU_PACK[:-1], CU_PACK[1:]):
+        for i in range(t1 - t0):
+            n = (i + 1) if causal else (t1 - t0)
+            for h in range(H):
+                want = v[t0:t0 + n, h // 2].mean(axis=0)
+                assert np.abs(O[t0 + i, h] - want).max() < 1e-15
+                assert lse[h, t0 + i] == math.log(n)
+    assert np.all(O[13:] == 0) and np.all(np.isnan(lse[:, 13:]))
+
+
+def test_varlen_sequences_are_independent():
+    """Changing every input row of one sequence leaves every other sequence's outputs as they
+    were, bit for bit."""
+    T, H, H_kv, d = 15, 2, 1, 4
+    q, k, v, _ = _packed(T, H, H_kv, d, 62)
+    O1, l1 = oracle.attention_fwd_varlen(q, k, v, np.array(CU_PACK), 0.5, True)
+    q2, k2, v2 = q.copy(), k.copy(), v.copy()
+    q2[3:8] += 1.0
+    k2[3:8] -= 2.0
+    v2[3:8] *= 3.0
+    O2, l2 = oracle.attention_fwd_varlen(q2, k2, v2, np.array(CU_PACK), 0.5, True)
+    other = np.r_[0:3, 8:13]
+    assert np.array_equal(O1[other], O2[other]) and np.array_equal(l1[:, other], l2[:, other])
+    assert not np.allclose(O1[3:8], O2[3:8])
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_gradients_match_central_differences(causal):
+    """Gradients on the packed layout (scatter of per-sequence, per-head pieces) against central
+    differences of the packed forward."""
+    cu = np.array([0, 2, 2, 5, 6])
+    T, H, H_kv, d = 7, 2, 1, 3
+    q, k, v, do = _packed(T, H, H_kv, d, 63)
+    grads = oracle.attention_bwd_varlen(q, k, v, do, cu, 0.8, causal)
+    h = 1e-6
+
+    def loss(q_, k_, v_):
+        O, _ = oracle.attention_fwd_varlen(q_, k_, v_, cu, 0.8, causal)
+        return float((O * do).sum())
+
+    for name, arr, grad in (("q", q, grads["dq"]), ("k", k, grads["dk"]), ("v", v, grads["dv"])):
+        fd = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            args = {"q": q.copy(), "k": k.copy(), "v": v.copy()}
+            args[name][idx] += h
+            lp = loss(args["q"], args["k"], args["v"])
+            args[name][idx] -= 2 * h
+            lm = loss(args["q"], args["k"], args["v"])
+            fd[idx] = (lp - lm) / (2 * h)
+        assert np.abs(fd - grad).max() <= 1e-6 * max(1.0, np.abs(grad).max()), name
+    assert np.all(grads["dq"][6] == 0) and np.all(grads["dk"][6] == 0)
+
+
+def test_varlen_rejects_offsets_outside_the_pack():
+    q, k, v, _ = _packed(5, 1, 1, 2, 64)
+    for cu in ([0, 3, 2], [0, 6], [-1, 2]):
+        with pytest.raises(ValueError):
+            oracle.attention_fwd_varlen(q, k, v, np.array(cu), 1.0, False)

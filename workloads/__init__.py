@@ -132,6 +132,65 @@ def make_inputs(w: Workload, with_grad: bool = True) -> Inputs:
     return Inputs(q, k, v, do, seqlens)
 
 
+@dataclasses.dataclass(frozen=True)
+class PackedWorkload:
+    """Variable-length sequences stored back to back ([T, H, d] with offsets cu_seqlens)."""
+
+    name: str
+    B: int
+    H: int
+    H_kv: int
+    d: int
+    causal: bool
+    seed: int
+    len_range: tuple[int, int] = (1, 512)    # inclusive range the lengths are drawn from
+    lengths: Optional[tuple[int, ...]] = None  # fixed lengths instead of drawn ones
+    std: float = 1.0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / (self.d ** 0.5)
+
+
+@dataclasses.dataclass
+class PackedInputs:
+    q: torch.Tensor           # bf16 [T, H, d], CPU
+    k: torch.Tensor           # bf16 [T, H_kv, d]
+    v: torch.Tensor
+    do: torch.Tensor          # bf16 [T, H, d]
+    cu_seqlens: torch.Tensor  # int32 [B + 1], CPU
+    max_seqlen: int
+
+
+def make_packed_inputs(w: PackedWorkload) -> PackedInputs:
+    """Packed recipe: the B lengths are drawn first as UniformInt[lo, hi] (unless fixed), then
+    Q, K, V, dO in that order as fp32 std * N(0, 1) over the T = sum(lengths) packed rows,
+    rounded to bf16."""
+    g = torch.Generator().manual_seed(w.seed)
+    if w.lengths is not None:
+        lens = [int(x) for x in w.lengths]
+        assert len(lens) == w.B
+    else:
+        lo, hi = w.len_range
+        lens = torch.randint(lo, hi + 1, (w.B,), generator=g, dtype=torch.int64).tolist()
+    cu = [0]
+    for n in lens:
+        cu.append(cu[-1] + n)
+    T = max(cu[-1], 1)
+
+    def draw(sh) -> torch.Tensor:
+        x = torch.randn(sh, generator=g, dtype=torch.float32)
+        if w.std != 1.0:
+            x.mul_(w.std)
+        return x.to(torch.bfloat16)
+
+    q = draw((T, w.H, w.d))
+    k = draw((T, w.H_kv, w.d))
+    v = draw((T, w.H_kv, w.d))
+    do = draw((T, w.H, w.d))
+    return PackedInputs(q, k, v, do, torch.tensor(cu, dtype=torch.int32), max(max(lens), 1))
+
+
 def seeded_sample(seed: int, population: int, count: int) -> list[int]:
     """A seeded subset of range(population), sorted; used to pick heads and rows to check."""
     g = torch.Generator().manual_seed(seed)
