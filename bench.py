@@ -70,9 +70,17 @@ def load_peaks() -> tuple[dict, str]:
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+KERNEL_SOURCES = {
+    "fa_fwd_kernel": ("fa_fwd.cu", "sm100.cuh", "fa_internal.h"),
+    "fa_bwd_kernel": ("fa_bwd.cu", "sm100.cuh", "fa_internal.h"),
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of the sources a kernel is compiled from (a recorded traffic figure is only valid
+    for the exact code it was measured on)."""
     h = hashlib.sha256()
-    for name in ("fa_bwd.cu", "fa_fwd.cu", "sm100.cuh", "fa_internal.h"):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "io_aware_exact_16_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -87,7 +95,7 @@ def dram_traffic(kernel: str, workload: str) -> float | None:
     except (OSError, ValueError):
         return None
     entry = data.get(kernel, {})
-    if entry.get("workload") != workload or entry.get("source_hash") != kernel_source_hash():
+    if entry.get("workload") != workload or entry.get("source_hash") != kernel_source_hash(kernel):
         return None
     return float(entry["dram_bytes_per_launch"])
 

@@ -325,13 +325,21 @@ __global__ void __launch_bounds__(512, 1)
     // Step it visits query head q_head(it) of the group (each head in turn) and query block
     // q_block(it) of that head; dK and dV accumulate over every step, so they sum over the
     // group's query heads.
+    // Each role walks the steps with a Step cursor (g = head of the group, r = step within the
+    // head) instead of dividing `it` by n_it_head: an integer divide by a runtime value needs a
+    // reciprocal on the MUFU unit, which the exponentials of the P phase saturate.
     const int n_it_head = n_q - i_start;
     const int n_it = G * n_it_head;
-    auto q_head = [&](int it) { return bh_first + it / n_it_head; };
-    auto q_block = [&](int it) {
-        const int r = it % n_it_head;
-        if (p.causal) return j + r;
-        const int i = j + r;
+    struct Step {
+        int g, r;
+    };
+    auto next_step = [&](Step s) {
+        return s.r + 1 == n_it_head ? Step{s.g + 1, 0} : Step{s.g, s.r + 1};
+    };
+    auto q_head = [&](Step s) { return bh_first + s.g; };
+    auto q_block = [&](Step s) {
+        const int i = j + s.r;
+        if (p.causal) return i;
         return i < n_q ? i : i - n_q;
     };
 
@@ -374,14 +382,15 @@ __global__ void __launch_bounds__(512, 1)
         // Named barriers have no timeout: every drain thread executes each of them, also after
         // a failed wait (`ok` then only skips the work).
         bool ok = true;
-        for (int it = 0; it < n_it; ++it) {
-            const int q0 = q_block(it) * C::BM;
+        Step st{0, 0};
+        for (int it = 0; it < n_it; ++it, st = next_step(st)) {
+            const int q0 = q_block(st) * C::BM;
             // fixed-point scale of query q0 + r (rows past N: scale 0), shared by the drain
             // warps; barrier 2 before the reads and again after the last read of the step
             {
                 const int q = q0 + r;
                 s_scale[r] =
-                    q < ext.Lq ? fixed_point_scale(p.dOnorm[(size_t)q_head(it) * p.N + q], factor) : 0.f;
+                    q < ext.Lq ? fixed_point_scale(p.dOnorm[(size_t)q_head(st) * p.N + q], factor) : 0.f;
             }
             named_barrier(2, 128);
             const float* sc = s_scale;
@@ -397,7 +406,7 @@ __global__ void __launch_bounds__(512, 1)
                 for (int q = 0; q < NV / 32; ++q) reg_fence32(v + 32 * q);
                 tc_fence_before();
                 mbar_arrive(bar_dqempty);           // B may take the next dP^T
-                int* acc = p.dq_acc + ((size_t)q_head(it) * p.N_pad + q0) * D;
+                int* acc = p.dq_acc + ((size_t)q_head(st) * p.N_pad + q0) * D;
                 if constexpr (D == 128) {
                     // dQ^T: lane = feature r, column = query e; a warp instruction covers 32
                     // consecutive features of one query row: one 128-byte line.
@@ -441,11 +450,12 @@ __global__ void __launch_bounds__(512, 1)
             tma_load_3d(smem + C::SMEM_V + c * C::CHUNK_BYTES, &tmV, bar_kv, c * 64, kv_y, kv_z);
         }
         int it = 0;
-        for (; it < n_it; ++it) {
+        Step st{0, 0};
+        for (; it < n_it; ++it, st = next_step(st)) {
             const int s = it % C::QST;
             const uint32_t ph = (it / C::QST) & 1;
-            const int q0 = q_block(it) * C::BM;
-            const int qh = q_head(it);
+            const int q0 = q_block(st) * C::BM;
+            const int qh = q_head(st);
             if (!mbar_wait(&bar_qempty[s], ph ^ 1, p.timeout_ns, abort_flag)) { fail(); break; }
             mbar_arrive_expect_tx(&bar_qfull[s], 2 * C::Q_TILE_BYTES);
             for (int c = 0; c < C::KCH; ++c) {
@@ -579,19 +589,19 @@ __global__ void __launch_bounds__(512, 1)
         // lse of query head bh_first + g, position q: lse[lse_base + g * lse_hstride + q].
         const size_t lse_hstride = packed ? (size_t)p.T : (size_t)p.N;
         const size_t lse_base = lse_of(packed, b, bh_first - b * p.H, p.H, p.N, p.T, ext.t0, 0);
-        auto load_vectors = [&](int it) {
-            const int q = q_block(it) * C::BM + (ct & 127);
-            const int g = it / n_it_head;  // head of the group
+        auto load_vectors = [&](Step st) {
+            const int q = q_block(st) * C::BM + (ct & 127);
             if (ct < 128)
-                staged = q < ext.Lq ? -p.lse[lse_base + (size_t)g * lse_hstride + q] * kLog2e
+                staged = q < ext.Lq ? -p.lse[lse_base + (size_t)st.g * lse_hstride + q] * kLog2e
                                     : -INFINITY;
-            else staged = q < ext.Lq ? p.Dvec[(size_t)(bh_first + g) * p.N + q] : 0.f;
+            else staged = q < ext.Lq ? p.Dvec[(size_t)q_head(st) * p.N + q] : 0.f;
         };
         auto store_vectors = [&](int it) {
             if (ct < 128) s_lse2[(it & 1) * C::BM + ct] = staged;
             else s_D[(it & 1) * C::BM + (ct - 128)] = staged;
         };
-        load_vectors(0);
+        Step st{0, 0};
+        load_vectors(st);
         store_vectors(0);
         named_barrier(1, 256);
 
@@ -599,10 +609,11 @@ __global__ void __launch_bounds__(512, 1)
         // after a failed (timed-out or aborted) wait; `ok` then only skips the work.
         bool ok = true;
         for (int it = 0; it < n_it; ++it) {
-            const int i = q_block(it);
+            const int i = q_block(st);
+            st = next_step(st);                      // the step of it + 1 from here on
             const float* lse2 = s_lse2 + (it & 1) * C::BM + 64 * h;
             const float* Dv = s_D + (it & 1) * C::BM + 64 * h;
-            if (it + 1 < n_it) load_vectors(it + 1);  // stored at the end of this iteration
+            if (it + 1 < n_it) load_vectors(st);   // stored at the end of this iteration
             const bool diag = p.causal && (i == j);
 
             // ---------------- P phase
