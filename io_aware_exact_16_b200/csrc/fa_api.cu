@@ -10,6 +10,11 @@
 #include "fa_internal.h"
 
 namespace fa {
+
+// fa_fwd_d256.cu: head dimension 256 (forward only).
+cudaError_t launch_fwd_d256(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const FwdParams& p, int B, cudaStream_t stream);
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -82,10 +87,11 @@ DeviceState* current_device(fa_status* st) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-fa_status check_common(int B, int H, int N, int d, float scale) {
+// d = 256 has a forward kernel only (`fwd`).
+fa_status check_common(int B, int H, int N, int d, float scale, bool fwd = false) {
     if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
     if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
-    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128 && !(fwd && d == 256)) return FA_ERR_UNSUPPORTED;
     if (B > 65535 || H > 65535) return FA_ERR_INVALID_ARG;
     const long long elems = (long long)B * H * N * d;
     if (elems >= (1ll << 31)) return FA_ERR_INVALID_ARG;
@@ -133,8 +139,8 @@ bool user_map(CUtensorMap* map, const void* base, int d, int B, int Hx, int N, i
 
 // Checks shared by the head-major and packed entry points; T = 0 for head-major.
 fa_status check_layout(int B, int H, int H_kv, int N, int d, float scale, const int* seqlens,
-                       const int* cu_seqlens, int T) {
-    fa_status st = check_common(B, H, N, d, scale);
+                       const int* cu_seqlens, int T, bool fwd) {
+    fa_status st = check_common(B, H, N, d, scale, fwd);
     if (st != FA_OK) return st;
     if (H_kv < 1 || H_kv > H || H % H_kv != 0) return FA_ERR_INVALID_ARG;
     if (seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u)) return FA_ERR_INVALID_ARG;
@@ -148,7 +154,7 @@ fa_status check_layout(int B, int H, int H_kv, int N, int d, float scale, const 
 fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                    int H_kv, int N, int d, float scale, int causal, const int* seqlens,
                    const int* cu_seqlens, int T, cudaStream_t stream) {
-    fa_status st = check_layout(B, H, H_kv, N, d, scale, seqlens, cu_seqlens, T);
+    fa_status st = check_layout(B, H, H_kv, N, d, scale, seqlens, cu_seqlens, T, true);
     if (st != FA_OK) return st;
     if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
@@ -174,7 +180,9 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
     p.timeout_ns = g_timeout_ns.load();
-    if (launch_fwd(d, tq, tk, tv, p, B, dev->num_sms, stream) != cudaSuccess) return FA_ERR_CUDA;
+    const cudaError_t e = d == 256 ? launch_fwd_d256(tq, tk, tv, p, B, stream)
+                                   : launch_fwd(d, tq, tk, tv, p, B, dev->num_sms, stream);
+    if (e != cudaSuccess) return FA_ERR_CUDA;
     return FA_OK;
 }
 
@@ -239,7 +247,7 @@ static fa_status bwd_impl(const void* q, const void* k, const void* v, const voi
                           int H, int H_kv, int N, int d, float scale, int causal,
                           const int* seqlens, const int* cu_seqlens, int T, void* workspace,
                           size_t workspace_bytes, cudaStream_t stream) {
-    fa_status st = check_layout(B, H, H_kv, N, d, scale, seqlens, cu_seqlens, T);
+    fa_status st = check_layout(B, H, H_kv, N, d, scale, seqlens, cu_seqlens, T, false);
     if (st != FA_OK) return st;
     if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dO) ||
