@@ -178,6 +178,35 @@ FA_API fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, cons
                                size_t workspace_bytes, fa_stream_t stream);
 
 /*
+ * Decode: a few new queries per sequence against a long key/value cache (token-by-token
+ * generation; FlashAttention (DE), "Spezialisierte Lösungen": FlashInfer's processing of the
+ * KV cache in streaming generation, FlashDecoding).  Forward only.
+ *   q, o           bf16 [B, H, Nq, d]        Nq >= 1 new queries per sequence
+ *   k_cache, v_cache bf16 [B, H_kv, N, d]    N = cache capacity; H % H_kv == 0 and query head h
+ *                                            reads cache head h / (H / H_kv)
+ *   lse            fp32 [B, H, Nq]           natural-log units
+ *   cache_lens     device int32 [B] valid cache rows L_b in [1, N] (rows >= L_b are ignored),
+ *                  or NULL for L_b = N; out-of-range values are clamped and reported.
+ *   causal         query i (0-based of Nq) is position L_b - Nq + i and sees keys
+ *                  j <= L_b - Nq + i (aligned to the end of the cache); a query that sees no
+ *                  key gets O = 0 and lse = -inf.
+ *   splits         key ranges per (sequence, cache head) computed by separate CTAs and merged
+ *                  by their log-sum-exp; 0 = fa_decode_num_splits(...).  The value is capped at
+ *                  the number of 128-key blocks of N.
+ *   workspace      device, 16-byte aligned, >= fa_decode_workspace_size(B, H, Nq, d, splits)
+ *                  bytes when splits > 1 (pass the splits the call will use); may be NULL
+ *                  when splits == 1.
+ * d in {64, 128, 256}.  The result is exact for every `splits` (up to rounding: different
+ * splits round differently; the same splits give identical bits).
+ */
+FA_API int fa_decode_num_splits(int B, int H, int H_kv, int Nq, int N, int d);
+FA_API size_t fa_decode_workspace_size(int B, int H, int Nq, int d, int splits);
+FA_API fa_status fa_fwd_decode(const void* q, const void* k_cache, const void* v_cache, void* o,
+                               float* lse, const int* cache_lens, int B, int H, int H_kv,
+                               int Nq, int N, int d, float scale, int causal, int splits,
+                               void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
  * fa_bwd_noalloc -- the backward pass without any device allocation.  The pages have no
  * counterpart of this entry point; it exists for callers that cannot allocate device memory:
  * a process that reserves its whole device-memory budget for its own pool up front, or a

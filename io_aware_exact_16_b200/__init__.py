@@ -6,7 +6,7 @@ device pointers and the current CUDA stream from PyTorch, and calls the C ABI in
 kernels; there is no CPU or PyTorch fallback.  If the library is missing or fails to load,
 importing this module raises ``ImportError``.
 
-Build the library with ``python -m io_aware_exact_16_b200.build``.
+Build the library with ``python io_aware_exact_16_b200/build.py``.
 """
 from __future__ import annotations
 
@@ -20,7 +20,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfa.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m io_aware_exact_16_b200.build`")
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python io_aware_exact_16_b200/build.py`")
 try:
     _lib = ctypes.CDLL(LIB_PATH)
 except OSError as exc:  # pragma: no cover
@@ -45,6 +45,13 @@ _lib.fa_fwd_varlen.restype = _i
 _lib.fa_bwd_varlen.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
                                _i, _i, ctypes.c_float, _i, _vp, ctypes.c_size_t, _vp]
 _lib.fa_bwd_varlen.restype = _i
+_lib.fa_decode_num_splits.argtypes = [_i, _i, _i, _i, _i, _i]
+_lib.fa_decode_num_splits.restype = _i
+_lib.fa_decode_workspace_size.argtypes = [_i, _i, _i, _i, _i]
+_lib.fa_decode_workspace_size.restype = ctypes.c_size_t
+_lib.fa_fwd_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                               ctypes.c_float, _i, _i, _vp, ctypes.c_size_t, _vp]
+_lib.fa_fwd_decode.restype = _i
 _lib.fa_bwd_workspace_size.argtypes = [_i, _i, _i, _i]
 _lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
 _lib.fa_check_device_error.argtypes = [_vp]
@@ -56,6 +63,7 @@ _lib.fa_status_string.restype = ctypes.c_char_p
 
 # Every symbol include/fa.h declares.
 EXPORTED = ("fa_fwd", "fa_bwd", "fa_fwd_gqa", "fa_bwd_gqa", "fa_fwd_varlen", "fa_bwd_varlen",
+            "fa_decode_num_splits", "fa_decode_workspace_size", "fa_fwd_decode",
             "fa_bwd_workspace_size",
             "fa_check_device_error", "fa_set_wait_timeout_ns", "fa_status_string",
             "fa_bwd_noalloc")
@@ -250,6 +258,55 @@ def backward_varlen(q, k, v, o, do, lse, cu_seqlens, max_seqlen: int, causal: bo
     if st != FA_OK:
         raise FAError(st, "fa_bwd_varlen")
     return dq, dk, dv
+
+
+def decode_num_splits(B: int, H: int, H_kv: int, Nq: int, N: int, d: int) -> int:
+    return int(_lib.fa_decode_num_splits(B, H, H_kv, Nq, N, d))
+
+
+def decode(q, k_cache, v_cache, cache_lens: Optional[torch.Tensor] = None, causal: bool = False,
+           scale: Optional[float] = None, splits: int = 0, out=None, lse=None,
+           workspace: Optional[torch.Tensor] = None):
+    """``fa_fwd_decode``: q [B, H, Nq, d] against k_cache, v_cache [B, H_kv, N, d] (valid rows
+    per sequence: cache_lens int32 [B], or all N).  Returns (O bf16 [B, H, Nq, d],
+    lse fp32 [B, H, Nq])."""
+    B, H, Nq, d = q.shape
+    dev = q.device
+    if k_cache.dim() != 4:
+        raise ValueError("k_cache must be [B, H_kv, N, d]")
+    H_kv, N = k_cache.shape[1], k_cache.shape[2]
+    if H_kv < 1 or H % H_kv != 0:
+        raise ValueError(f"cache heads {H_kv} must divide query heads {H}")
+    _check_qkv("q", q, (B, H, Nq, d), dev)
+    for name, t in (("k_cache", k_cache), ("v_cache", v_cache)):
+        _check_qkv(name, t, (B, H_kv, N, d), dev)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check_qkv("out", out, (B, H, Nq, d), dev)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=dev)
+    elif lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, Nq) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 tensor [B, H, Nq]")
+    if splits == 0:
+        splits = decode_num_splits(B, H, H_kv, Nq, N, d)
+    nblk = (N + 127) // 128
+    splits = max(1, min(int(splits), nblk))
+    bps = (nblk + splits - 1) // splits
+    splits = (nblk + bps - 1) // bps
+    need = int(_lib.fa_decode_workspace_size(B, H, Nq, d, splits))
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    sc = float(scale) if scale is not None else 1.0 / (d ** 0.5)
+    st = _lib.fa_fwd_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                            out.data_ptr(), lse.data_ptr(), _seqlens_ptr(cache_lens, B, dev), B, H,
+                            H_kv, Nq, N, d, sc, int(bool(causal)), splits, ws_ptr, ws_bytes,
+                            _stream_handle(dev))
+    if st != FA_OK:
+        raise FAError(st, "fa_fwd_decode")
+    return out, lse
 
 
 def check_device_error(device: Optional[torch.device] = None) -> int:

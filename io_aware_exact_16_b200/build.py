@@ -1,7 +1,8 @@
 """Builds the CUDA library ``libfa.so`` in-tree for sm_100a with nvcc.
 
 The library is the C ABI of ``include/fa.h``; the Python binding in this package loads it
-with ctypes.  Run ``python -m io_aware_exact_16_b200.build`` (or call ``build()``).
+with ctypes.  Run ``python io_aware_exact_16_b200/build.py`` (a plain script: importing the
+package first would try to load the library it builds).
 """
 from __future__ import annotations
 
@@ -13,8 +14,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 SO = os.path.join(HERE, "libfa.so")
-SOURCES = ["fa_api.cu", "fa_fwd.cu", "fa_bwd.cu", "fa_bwd_noalloc.cu", "fa_fwd_d256.cu"]
-HEADERS = ["fa_internal.h", "sm100.cuh", os.path.join("..", "..", "include", "fa.h")]
+SOURCES = ["fa_api.cu", "fa_fwd.cu", "fa_bwd.cu", "fa_bwd_noalloc.cu", "fa_fwd_d256.cu", "fa_decode.cu"]
+HEADERS = ["fa_internal.h", "fa_decode.h", "sm100.cuh", os.path.join("..", "..", "include", "fa.h")]
 
 
 def nvcc() -> str:

@@ -7,6 +7,7 @@
 #include <cmath>
 #include <mutex>
 
+#include "fa_decode.h"
 #include "fa_internal.h"
 
 namespace fa {
@@ -186,6 +187,36 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
     return FA_OK;
 }
 
+// Split-KV decode: the number of key ranges that minimises (waves of CTAs) x (128-key blocks
+// per CTA + 1 for its fixed cost), preferring fewer ranges on ties.
+int decode_splits(int B, int H_kv, int n_mt, int N, int num_sms) {
+    const int nblk = (N + 127) / 128;
+    const long long base = (long long)B * H_kv * n_mt;
+    int best = 1;
+    long long best_cost = -1;
+    for (int s = 1; s <= nblk && s <= 256; ++s) {
+        const int bps = (nblk + s - 1) / s;
+        if ((nblk + bps - 1) / bps != s) continue;  // same ranges as a smaller s
+        const long long waves = (base * s + num_sms - 1) / num_sms;
+        const long long cost = waves * (bps + 1);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = s;
+        }
+    }
+    return best;
+}
+
+fa_status check_decode(int B, int H, int H_kv, int Nq, int N, int d, float scale, int splits) {
+    if (B < 1 || H < 1 || H_kv < 1 || Nq < 1 || N < 1 || splits < 0) return FA_ERR_INVALID_ARG;
+    if (H % H_kv != 0 || B > 65535 || H > 65535) return FA_ERR_INVALID_ARG;
+    if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+    if ((long long)B * H * Nq * d >= (1ll << 31) || (long long)B * H_kv * N * d >= (1ll << 31))
+        return FA_ERR_INVALID_ARG;
+    return FA_OK;
+}
+
 }  // namespace
 }  // namespace fa
 
@@ -328,6 +359,87 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  size_t workspace_bytes, fa_stream_t stream) {
     return fa_bwd_gqa(q, k, v, o, dO, lse, dq, dk, dv, B, H, H, N, d, scale, causal, seqlens,
                       workspace, workspace_bytes, stream);
+}
+
+int fa_decode_num_splits(int B, int H, int H_kv, int Nq, int N, int d) {
+    if (check_decode(B, H, H_kv, Nq, N, d, 1.0f, 0) != FA_OK) return 0;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+            sms = v;
+    }
+    const int n_mt = ((H / H_kv) * Nq + 127) / 128;
+    return decode_splits(B, H_kv, n_mt, N, sms);
+}
+
+size_t fa_decode_workspace_size(int B, int H, int Nq, int d, int splits) {
+    if (B < 1 || H < 1 || Nq < 1 || splits < 1 || (d != 64 && d != 128 && d != 256)) return 0;
+    if (splits == 1) return 0;
+    const size_t rows = (size_t)B * H * Nq;
+    const size_t o_bytes = ((size_t)splits * rows * d * sizeof(float) + 255) / 256 * 256;
+    return o_bytes + (size_t)splits * rows * sizeof(float);
+}
+
+fa_status fa_fwd_decode(const void* q, const void* k_cache, const void* v_cache, void* o,
+                        float* lse, const int* cache_lens, int B, int H, int H_kv, int Nq, int N,
+                        int d, float scale, int causal, int splits, void* workspace,
+                        size_t workspace_bytes, fa_stream_t stream) {
+    fa_status st = check_decode(B, H, H_kv, Nq, N, d, scale, splits);
+    if (st != FA_OK) return st;
+    if (!q || !k_cache || !v_cache || !o || !lse) return FA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+        !aligned16(lse))
+        return FA_ERR_INVALID_ARG;
+    if (cache_lens && (reinterpret_cast<uintptr_t>(cache_lens) & 3u)) return FA_ERR_INVALID_ARG;
+    DeviceState* dev = current_device(&st);
+    if (!dev) return st;
+
+    const int G = H / H_kv;
+    const int n_mt = (G * Nq + 127) / 128;
+    const int nblk = (N + 127) / 128;
+    if (splits == 0) splits = decode_splits(B, H_kv, n_mt, N, dev->num_sms);
+    if (splits > nblk) splits = nblk;
+    const int bps = (nblk + splits - 1) / splits;
+    splits = (nblk + bps - 1) / bps;  // ranges that actually hold keys
+    if ((long long)H_kv * n_mt > 65535) return FA_ERR_INVALID_ARG;  // grid.y
+
+    DecodeParams p{};
+    p.o = o;
+    p.lse = lse;
+    if (splits > 1) {
+        const size_t need = fa_decode_workspace_size(B, H, Nq, d, splits);
+        if (!workspace || !aligned16(workspace) || workspace_bytes < need)
+            return FA_ERR_WORKSPACE;
+        const size_t rows = (size_t)B * H * Nq;
+        p.o_part = static_cast<float*>(workspace);
+        p.lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                              ((size_t)splits * rows * d * sizeof(float) + 255) /
+                                                  256 * 256);
+    }
+    p.cache_lens = cache_lens;
+    p.err = dev->err_flag;
+    p.B = B;
+    p.H = H;
+    p.H_kv = H_kv;
+    p.G = G;
+    p.Nq = Nq;
+    p.N = N;
+    p.n_mtiles = n_mt;
+    p.splits = splits;
+    p.blocks_per_split = bps;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.causal = causal ? 1 : 0;
+    p.timeout_ns = g_timeout_ns.load();
+
+    CUtensorMap tq, tk, tv;
+    if (!make_bf16_map(&tq, q, d, G * Nq, B * H_kv, 128) ||
+        !make_bf16_map(&tk, k_cache, d, N, B * H_kv, 128) ||
+        !make_bf16_map(&tv, v_cache, d, N, B * H_kv, 128))
+        return FA_ERR_CUDA;
+    if (launch_decode(d, tq, tk, tv, p, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return FA_ERR_CUDA;
+    return FA_OK;
 }
 
 fa_status fa_check_device_error(fa_stream_t stream) {

@@ -301,3 +301,37 @@ def attention_bwd_varlen(q, k, v, do, cu_seqlens, scale: float, causal: bool):
             out["dk"][t0:t1, kv[h]] += r["dk"]
             out["dv"][t0:t1, kv[h]] += r["dv"]
     return out
+
+
+def attention_decode(q, k_cache, v_cache, scale: float, causal: bool, cache_lens=None):
+    """Decode: Nq new queries per sequence, q [B, H, Nq, d], against a key/value cache
+    k, v [B, H_kv, N, d] of which sequence b uses its first L_b rows (all N without
+    ``cache_lens``); query head h reads cache head h // (H / H_kv).  Query i is position
+    L_b - Nq + i of its sequence; causal, it sees keys j <= L_b - Nq + i, otherwise all j < L_b.
+    The plain definition per (b, h, i) in fp64: scores s_j = scale * q_i . k_j over the visible
+    keys, lse = m + ln sum exp(s_j - m), O = sum_j exp(s_j - lse) v_j (two passes, matrix
+    products from numpy).  A query that sees no key gets O = 0 and lse = -inf."""
+    q, k, v = as_f64(q), as_f64(k_cache), as_f64(v_cache)
+    B, H, Nq, d = q.shape
+    H_kv, N = k.shape[1], k.shape[2]
+    kv = _kv_index(H, H_kv)
+    Ls = _lengths(cache_lens, B, N)
+    O = np.zeros((B, H, Nq, d), np.float64)
+    lse = np.full((B, H, Nq), -np.inf, np.float64)
+    for b in range(B):
+        L = Ls[b]
+        if not 1 <= L <= N:
+            raise ValueError("cache length outside [1, N]")
+        for h in range(H):
+            s = scale * (q[b, h] @ k[b, kv[h], :L].T)  # [Nq, L]
+            for i in range(Nq):
+                lim = min(L, L - Nq + i + 1) if causal else L
+                if lim <= 0:
+                    continue
+                row = s[i, :lim]
+                m = row.max()
+                e = np.exp(row - m)
+                tot = e.sum()
+                lse[b, h, i] = m + np.log(tot)
+                O[b, h, i] = (e / tot) @ v[b, kv[h], :lim]
+    return O, lse

@@ -478,3 +478,75 @@ def test_varlen_rejects_offsets_outside_the_pack():
     for cu in ([0, 3, 2], [0, 6], [-1, 2]):
         with pytest.raises(ValueError):
             oracle.attention_fwd_varlen(q, k, v, np.array(cu), 1.0, False)
+
+
+# ------------------------------------------------------------------ decode (KV cache)
+def _decode_inputs(B, H, H_kv, Nq, N, d, seed):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn((B, H, Nq, d), generator=g).to(torch.bfloat16).double().numpy()
+    k = torch.randn((B, H_kv, N, d), generator=g).to(torch.bfloat16).double().numpy()
+    v = torch.randn((B, H_kv, N, d), generator=g).to(torch.bfloat16).double().numpy()
+    return q, k, v
+
+
+def test_decode_with_all_positions_as_queries_is_causal_self_attention():
+    """Nq = L: the end-aligned causal mask becomes the ordinary j <= i mask, so the decode
+    definition must equal the pinned C oracle's causal self-attention on the same rows."""
+    q, k, v = _decode_inputs(1, 2, 2, 9, 9, 5, 71)
+    O, lse = oracle.attention_decode(q, k, v, 0.4, True)
+    for h in range(2):
+        O_ref, lse_ref = oracle.head_fwd(q[0, h], k[0, h], v[0, h], 0.4, True)
+        assert np.abs(O[0, h] - O_ref).max() < 1e-13
+        assert np.abs(lse[0, h] - lse_ref).max() < 1e-13
+
+
+def test_decode_zero_queries_average_the_visible_end_aligned_cache_rows():
+    """Q = 0: query i averages value rows 0 .. lim-1 with lim = L - Nq + i + 1 (causal) or L,
+    lse = ln(lim) exactly; cache rows >= L never enter; a query seeing nothing gets (0, -inf)."""
+    B, H, H_kv, Nq, N, d = 2, 4, 2, 3, 12, 3
+    _, k, v = _decode_inputs(B, H, H_kv, Nq, N, d, 72)
+    q = np.zeros((B, H, Nq, d))
+    lens = [7, 2]
+    for causal in (False, True):
+        O, lse = oracle.attention_decode(q, k, v, 1.3, causal, lens)
+        for b in range(B):
+            L = lens[b]
+            for h in range(H):
+                for i in range(Nq):
+                    lim = min(L, L - Nq + i + 1) if causal else L
+                    if lim <= 0:
+                        assert np.all(O[b, h, i] == 0) and lse[b, h, i] == -np.inf
+                        continue
+                    assert np.abs(O[b, h, i] - v[b, h // 2, :lim].mean(axis=0)).max() < 1e-15
+                    assert lse[b, h, i] == math.log(lim)
+
+
+def test_decode_merging_key_ranges_by_lse_gives_the_whole_result():
+    """The split-KV identity the GPU combine relies on, checked on the definition: attention
+    over the cache rows [0, a) and [a, L) separately, merged by lse = log(e^lse1 + e^lse2) and
+    O = e^(lse1 - lse) O1 + e^(lse2 - lse) O2, equals attention over [0, L)."""
+    q, k, v = _decode_inputs(1, 2, 1, 2, 20, 4, 73)
+    O, lse = oracle.attention_decode(q, k, v, 0.5, False)
+    a = 7
+    O1, l1 = oracle.attention_decode(q, k[:, :, :a], v[:, :, :a], 0.5, False)
+    O2, l2 = oracle.attention_decode(q, k[:, :, a:], v[:, :, a:], 0.5, False)
+    lm = np.logaddexp(l1, l2)
+    Om = np.exp(l1 - lm)[..., None] * O1 + np.exp(l2 - lm)[..., None] * O2
+    assert np.abs(lm - lse).max() < 1e-13 and np.abs(Om - O).max() < 1e-13
+
+
+def test_decode_single_query_causal_equals_non_causal_and_torch():
+    """Nq = 1 sees the whole valid cache with or without the causal flag; both agree with
+    torch float64 scaled_dot_product_attention on the valid rows."""
+    q, k, v = _decode_inputs(2, 4, 1, 1, 10, 6, 74)
+    lens = [10, 4]
+    Oc, lc = oracle.attention_decode(q, k, v, 0.3, True, lens)
+    On, ln_ = oracle.attention_decode(q, k, v, 0.3, False, lens)
+    assert np.array_equal(Oc, On) and np.array_equal(lc, ln_)
+    for b in range(2):
+        L = lens[b]
+        for h in range(4):
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                torch.from_numpy(q[b, h][None]), torch.from_numpy(k[b, 0, :L][None]),
+                torch.from_numpy(v[b, 0, :L][None]), scale=0.3)[0]
+            assert np.abs(On[b, h] - ref.numpy()).max() < 1e-12
