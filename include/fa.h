@@ -207,6 +207,23 @@ FA_API fa_status fa_fwd_decode(const void* q, const void* k_cache, const void* v
                                void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
 /*
+ * FP8 forward (FlashAttention-3's FP8 mode; Russian article, "FlashAttention-3 (2024)").
+ * q, k, v hold OCP FP8 E4M3 codes ("fn" variant, one byte each), layout as fa_fwd_gqa with
+ * d = 128 only: q [B, H, N, 128], k, v [B, H_kv, N, 128].  The values they stand for are
+ * code * descale with per-(batch, head) fp32 factors q_descale [B, H], k_descale [B, H_kv],
+ * v_descale [B, H_kv] (device arrays, 4-byte aligned; NULL means 1).  O (bf16 [B, H, N, 128])
+ * and lse (fp32 [B, H, N]) are those of exact attention of the dequantised values, up to the
+ * rounding of the probabilities to e4m3 before the P V product: |O - O_exact| is bounded per
+ * element by 2^-4 * sum_j P_ij |v_jc| + 2^-14 * sum_{visible j} |v_jc| (relative e4m3 rounding,
+ * and absolute underflow of probabilities below 2^-14 of the row's largest) plus bf16 output
+ * rounding.  Masks, seqlens and errors as fa_fwd.  d != 128: FA_ERR_UNSUPPORTED.
+ */
+FA_API fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, const float* q_descale,
+                            const float* k_descale, const float* v_descale, void* o, float* lse,
+                            int B, int H, int H_kv, int N, int d, float scale, int causal,
+                            const int* seqlens, fa_stream_t stream);
+
+/*
  * fa_bwd_noalloc -- the backward pass without any device allocation.  The pages have no
  * counterpart of this entry point; it exists for callers that cannot allocate device memory:
  * a process that reserves its whole device-memory budget for its own pool up front, or a

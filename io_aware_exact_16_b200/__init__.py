@@ -52,6 +52,9 @@ _lib.fa_decode_workspace_size.restype = ctypes.c_size_t
 _lib.fa_fwd_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
                                ctypes.c_float, _i, _i, _vp, ctypes.c_size_t, _vp]
 _lib.fa_fwd_decode.restype = _i
+_lib.fa_fwd_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
+                            ctypes.c_float, _i, _vp, _vp]
+_lib.fa_fwd_fp8.restype = _i
 _lib.fa_bwd_workspace_size.argtypes = [_i, _i, _i, _i]
 _lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
 _lib.fa_check_device_error.argtypes = [_vp]
@@ -64,7 +67,7 @@ _lib.fa_status_string.restype = ctypes.c_char_p
 # Every symbol include/fa.h declares.
 EXPORTED = ("fa_fwd", "fa_bwd", "fa_fwd_gqa", "fa_bwd_gqa", "fa_fwd_varlen", "fa_bwd_varlen",
             "fa_decode_num_splits", "fa_decode_workspace_size", "fa_fwd_decode",
-            "fa_bwd_workspace_size",
+            "fa_fwd_fp8", "fa_bwd_workspace_size",
             "fa_check_device_error", "fa_set_wait_timeout_ns", "fa_status_string",
             "fa_bwd_noalloc")
 
@@ -258,6 +261,50 @@ def backward_varlen(q, k, v, o, do, lse, cu_seqlens, max_seqlen: int, causal: bo
     if st != FA_OK:
         raise FAError(st, "fa_bwd_varlen")
     return dq, dk, dv
+
+
+def _descale_ptr(t: Optional[torch.Tensor], shape, device) -> Optional[int]:
+    if t is None:
+        return None
+    if t.dtype != torch.float32 or tuple(t.shape) != tuple(shape) or t.device != device:
+        raise ValueError(f"descale factors must be float32 {tuple(shape)} on {device}")
+    if not t.is_contiguous():
+        raise ValueError("descale factors must be contiguous")
+    return t.data_ptr()
+
+
+def forward_fp8(q, k, v, q_descale=None, k_descale=None, v_descale=None, causal: bool = False,
+                seqlens: Optional[torch.Tensor] = None, scale: Optional[float] = None,
+                out=None, lse=None):
+    """``fa_fwd_fp8``: q [B, H, N, 128], k, v [B, H_kv, N, 128] as torch.float8_e4m3fn codes
+    with per-(batch, head) float32 descale factors ([B, H], [B, H_kv], [B, H_kv]; None = 1).
+    Returns (O bf16 [B, H, N, 128], lse fp32 [B, H, N])."""
+    B, H, N, d = q.shape
+    dev = q.device
+    H_kv = k.shape[1]
+    if H_kv < 1 or H % H_kv != 0:
+        raise ValueError(f"key/value heads {H_kv} must divide query heads {H}")
+    for name, t, sh in (("q", q, (B, H, N, d)), ("k", k, (B, H_kv, N, d)),
+                        ("v", v, (B, H_kv, N, d))):
+        if t.dtype != torch.float8_e4m3fn:
+            raise TypeError(f"{name} must be float8_e4m3fn, got {t.dtype}")
+        if tuple(t.shape) != sh or t.device != dev or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous {sh} tensor on {dev}")
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    else:
+        _check_qkv("out", out, (B, H, N, d), dev)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    sc = float(scale) if scale is not None else 1.0 / (d ** 0.5)
+    st = _lib.fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                         _descale_ptr(q_descale, (B, H), dev), _descale_ptr(k_descale, (B, H_kv), dev),
+                         _descale_ptr(v_descale, (B, H_kv), dev), out.data_ptr(), lse.data_ptr(),
+                         B, H, H_kv, N, d, sc, int(bool(causal)), _seqlens_ptr(seqlens, B, dev),
+                         _stream_handle(dev))
+    if st != FA_OK:
+        raise FAError(st, "fa_fwd_fp8")
+    return out, lse
 
 
 def decode_num_splits(B: int, H: int, H_kv: int, Nq: int, N: int, d: int) -> int:

@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "fa_decode.h"
+#include "fa_fwd_fp8.h"
 #include "fa_internal.h"
 
 namespace fa {
@@ -126,6 +127,18 @@ bool make_bf16_map_packed(CUtensorMap* map, const void* base, int d, int Hx, int
     cuuint32_t estr[3] = {1, 1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_fp8_map(CUtensorMap* map, const void* base, int N, int BHx) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {128, (cuuint64_t)N, (cuuint64_t)BHx};
+    cuuint64_t strides[2] = {128, (cuuint64_t)N * 128};
+    cuuint32_t box[3] = {128, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -359,6 +372,46 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  size_t workspace_bytes, fa_stream_t stream) {
     return fa_bwd_gqa(q, k, v, o, dO, lse, dq, dk, dv, B, H, H, N, d, scale, causal, seqlens,
                       workspace, workspace_bytes, stream);
+}
+
+fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, const float* q_descale,
+                     const float* k_descale, const float* v_descale, void* o, float* lse, int B,
+                     int H, int H_kv, int N, int d, float scale, int causal, const int* seqlens,
+                     fa_stream_t stream) {
+    fa_status st = check_common(B, H, N, d, scale);
+    if (st != FA_OK) return st;
+    if (d != 128) return FA_ERR_UNSUPPORTED;
+    if (H_kv < 1 || H_kv > H || H % H_kv != 0) return FA_ERR_INVALID_ARG;
+    if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return FA_ERR_INVALID_ARG;
+    for (const void* ptr : {(const void*)q_descale, (const void*)k_descale,
+                            (const void*)v_descale, (const void*)seqlens})
+        if (ptr && (reinterpret_cast<uintptr_t>(ptr) & 3u)) return FA_ERR_INVALID_ARG;
+    DeviceState* dev = current_device(&st);
+    if (!dev) return st;
+
+    CUtensorMap tq, tk, tv;
+    if (!make_fp8_map(&tq, q, N, B * H) || !make_fp8_map(&tk, k, N, B * H_kv) ||
+        !make_fp8_map(&tv, v, N, B * H_kv))
+        return FA_ERR_CUDA;
+    Fp8Params p{};
+    p.o = o;
+    p.lse = lse;
+    p.seqlens = seqlens;
+    p.q_descale = q_descale;
+    p.k_descale = k_descale;
+    p.v_descale = v_descale;
+    p.err = dev->err_flag;
+    p.H = H;
+    p.N = N;
+    p.H_kv = H_kv;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.causal = causal ? 1 : 0;
+    p.timeout_ns = g_timeout_ns.load();
+    if (launch_fwd_fp8(tq, tk, tv, p, B, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return FA_ERR_CUDA;
+    return FA_OK;
 }
 
 int fa_decode_num_splits(int B, int H, int H_kv, int Nq, int N, int d) {

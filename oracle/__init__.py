@@ -335,3 +335,34 @@ def attention_decode(q, k_cache, v_cache, scale: float, causal: bool, cache_lens
                 lse[b, h, i] = m + np.log(tot)
                 O[b, h, i] = (e / tot) @ v[b, kv[h], :lim]
     return O, lse
+
+
+def decode_e4m3(codes) -> np.ndarray:
+    """Exact values of e4m3 (OCP FP8 E4M3, "fn" variant) codes, from the bit fields: sign bit,
+    4-bit exponent with bias 7, 3-bit mantissa; exponent 0 is subnormal (m/8 * 2^-6); the
+    all-ones pattern S.1111.111 is NaN; there are no infinities."""
+    if hasattr(codes, "detach"):  # a torch tensor of float8 codes: read its raw bytes
+        import torch
+        codes = codes.detach().cpu().contiguous().view(torch.uint8).numpy()
+    c = np.asarray(codes, dtype=np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    val = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * 2.0 ** (e - 7.0))
+    val = np.where((e == 0xF) & (m == 0x7), np.nan, val)
+    return sign * val
+
+
+def dequantize_fp8(codes, descale) -> np.ndarray:
+    """code * descale per (batch, head), exact in fp64: codes [B, Hx, N, d], descale [B, Hx]."""
+    return decode_e4m3(codes) * as_f64(descale)[:, :, None, None]
+
+
+def attention_fwd_fp8(q, k, v, q_descale, k_descale, v_descale, scale: float, causal: bool,
+                      seqlens=None):
+    """FP8 attention (FlashAttention-3's FP8 mode; Russian article, "FlashAttention-3 (2024)"):
+    the quantised inputs stand for the values code * descale, and the result is the exact
+    attention of those values (``attention_fwd_gqa`` in fp64).  The GPU's own rounding of P to
+    e4m3 is an approximation of this; its error bound lives with the parity tests."""
+    return attention_fwd_gqa(dequantize_fp8(q, q_descale), dequantize_fp8(k, k_descale),
+                             dequantize_fp8(v, v_descale), scale, causal, seqlens)

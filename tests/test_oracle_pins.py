@@ -550,3 +550,42 @@ def test_decode_single_query_causal_equals_non_causal_and_torch():
                 torch.from_numpy(q[b, h][None]), torch.from_numpy(k[b, 0, :L][None]),
                 torch.from_numpy(v[b, 0, :L][None]), scale=0.3)[0]
             assert np.abs(On[b, h] - ref.numpy()).max() < 1e-12
+
+
+# ------------------------------------------------------------------ FP8 (e4m3) inputs
+def test_e4m3_decoding_follows_the_bit_fields():
+    """Hand-decoded codes: 0x38 = 2^0 = 1, 0x7E = 1.75 * 2^8 = 448 (largest finite),
+    0x01 = 2^-9 (smallest subnormal), 0x08 = 2^-6 (smallest normal), 0x07 = 7/8 * 2^-6,
+    0xC5 = -(1 + 5/8) * 2 = -3.25, 0x7F = NaN."""
+    codes = np.array([0x38, 0x7E, 0x01, 0x08, 0x07, 0xC5, 0x7F, 0x00, 0x80])
+    got = oracle.decode_e4m3(codes)
+    want = [1.0, 448.0, 2.0 ** -9, 2.0 ** -6, 7 / 8 * 2.0 ** -6, -3.25, np.nan, 0.0, -0.0]
+    np.testing.assert_array_equal(got, np.array(want))
+
+
+def test_e4m3_decoding_agrees_with_torch_on_every_finite_code():
+    """All 254 finite codes against torch's float8_e4m3fn -> float64 conversion."""
+    codes = torch.arange(256, dtype=torch.uint8)
+    mine = oracle.decode_e4m3(codes.numpy())
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    finite = ~np.isnan(ref)
+    assert finite.sum() == 254
+    np.testing.assert_array_equal(mine[finite], ref[finite])
+    assert np.isnan(mine[~finite]).all()
+
+
+def test_fp8_attention_is_attention_of_the_dequantised_values():
+    """Scaling a head's descale by 2 and halving its codes' values is the same input; the FP8
+    oracle must see only code * descale (K descale folded into scores, V into O)."""
+    import workloads
+    w = workloads.custom(1, 2, 20, 8, True, seed=81)
+    f = workloads.make_fp8_inputs(w)
+    O, lse = oracle.attention_fwd_fp8(f.q, f.k, f.v, f.q_descale, f.k_descale, f.v_descale,
+                                      0.35, True)
+    q = oracle.decode_e4m3(f.q) * f.q_descale.double().numpy()[:, :, None, None]
+    k = oracle.decode_e4m3(f.k) * f.k_descale.double().numpy()[:, :, None, None]
+    v = oracle.decode_e4m3(f.v) * f.v_descale.double().numpy()[:, :, None, None]
+    O2, lse2 = oracle.attention_fwd_gqa(q, k, 2.0 * v, 0.35, True)
+    assert np.abs(2.0 * O - O2).max() < 1e-12 and np.abs(lse - lse2).max() == 0.0
+    # the quantised values stay within one e4m3 step (2^-3 relative) of the fp32 draws
+    assert np.all(np.abs(f.q.float().abs().numpy()) <= 448.0)

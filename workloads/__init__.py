@@ -191,6 +191,49 @@ def make_packed_inputs(w: PackedWorkload) -> PackedInputs:
     return PackedInputs(q, k, v, do, torch.tensor(cu, dtype=torch.int32), max(max(lens), 1))
 
 
+E4M3_MAX = 448.0
+
+
+@dataclasses.dataclass
+class FP8Inputs:
+    q: torch.Tensor          # float8_e4m3fn [B, H, N, d], CPU (codes)
+    k: torch.Tensor          # float8_e4m3fn [B, H_kv, N, d]
+    v: torch.Tensor
+    q_descale: torch.Tensor  # fp32 [B, H]:    q = code * q_descale
+    k_descale: torch.Tensor  # fp32 [B, H_kv]
+    v_descale: torch.Tensor  # fp32 [B, H_kv]
+    seqlens: Optional[torch.Tensor]
+
+
+def _quantize_per_head(x: torch.Tensor) -> tuple[torch.Tensor, torch.Tensor]:
+    """Per-(batch, head) scaling to the e4m3 range: descale = amax / 448, code =
+    e4m3(x / descale) (round to nearest even, clamped to +-448)."""
+    amax = x.abs().amax(dim=(2, 3)).clamp_min(1e-12)
+    descale = (amax / E4M3_MAX).to(torch.float32)
+    codes = (x / descale[:, :, None, None]).clamp(-E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn)
+    return codes, descale
+
+
+def make_fp8_inputs(w: Workload) -> FP8Inputs:
+    """FP8 recipe: the workload's fp32 draws (same generator order as ``make_inputs``: lengths,
+    then Q, K, V), each head quantised to e4m3 codes with a per-head descale factor."""
+    g = torch.Generator().manual_seed(w.seed)
+    seqlens = None
+    if w.pad_range is not None:
+        lo, hi = w.pad_range
+        seqlens = torch.randint(lo, hi + 1, (w.B,), generator=g, dtype=torch.int64).to(torch.int32)
+
+    def draw(sh) -> torch.Tensor:
+        x = torch.randn(sh, generator=g, dtype=torch.float32)
+        return x.mul_(w.std) if w.std != 1.0 else x
+
+    q = draw((w.B, w.H, w.N, w.d))
+    k = draw((w.B, w.kv_heads, w.N, w.d))
+    v = draw((w.B, w.kv_heads, w.N, w.d))
+    (qc, qd), (kc, kd), (vc, vd) = (_quantize_per_head(t) for t in (q, k, v))
+    return FP8Inputs(qc, kc, vc, qd, kd, vd, seqlens)
+
+
 def seeded_sample(seed: int, population: int, count: int) -> list[int]:
     """A seeded subset of range(population), sorted; used to pick heads and rows to check."""
     g = torch.Generator().manual_seed(seed)
