@@ -8,6 +8,7 @@ B = 16384 / N = 4 per GPU (the size at which the throughput targets are stated).
 FLOP accounting: forward 4*B*H*N^2*d (halved when causal), backward 2.5x the forward.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py --row fwd-d256|fwd-fp8|decode|varlen [...]   (the further entry points)
 
 With N > 1 launch one process per GPU with torch.distributed.run; each rank runs its own
 batch of the same shape (weak scaling, no collective on the data path) and rank 0 prints one
@@ -45,6 +46,9 @@ WORKLOADS = {
     "sweep-N4096-H32-d64": lambda: workloads.sweep(4096, 32, 64, False),
     "gpt2-small": workloads.gpt2_small,
     "bert-large-padded": workloads.bert_large_padded,
+    # grouped-query attention: 32 query heads over 8 key/value heads
+    "gqa-N4096-H32-kv8-d128": lambda: workloads.Workload(
+        "gqa non-causal B2 H32 Hkv8 N4096 d128", 2, 32, 4096, 128, False, 1040, H_kv=8),
 }
 DEFAULT_WORKLOAD = "sweep-N4096-H16-d128"
 
@@ -73,6 +77,9 @@ def load_peaks() -> tuple[dict, str]:
 KERNEL_SOURCES = {
     "fa_fwd_kernel": ("fa_fwd.cu", "sm100.cuh", "fa_internal.h"),
     "fa_bwd_kernel": ("fa_bwd.cu", "sm100.cuh", "fa_internal.h"),
+    "fa_fwd_d256_kernel": ("fa_fwd_d256.cu", "sm100.cuh", "fa_internal.h"),
+    "fa_fwd_fp8_kernel": ("fa_fwd_fp8.cu", "fa_fwd_fp8.h", "sm100.cuh", "fa_internal.h"),
+    "fa_decode_kernel": ("fa_decode.cu", "fa_decode.h", "sm100.cuh", "fa_internal.h"),
 }
 
 
@@ -175,7 +182,7 @@ class ClockSampler:
 def rank_workload(w: workloads.Workload, rank: int) -> workloads.Workload:
     """The batch rank `rank` processes: same shape, its own seed (independent batches)."""
     return workloads.Workload(w.name, w.B, w.H, w.N, w.d, w.causal, w.seed + 7919 * rank, w.std,
-                              w.pad_range)
+                              w.pad_range, H_kv=w.H_kv)
 
 
 def reduce_max(values: list[float], world: int, device=None) -> list[float]:
@@ -222,8 +229,12 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
         if world > 1:
             torch.distributed.barrier()
 
-    # ---- timed region: per-pass CUDA events on the launching stream
+    # ---- timed region: per-pass CUDA events on the launching stream, plus events the library
+    # records right around the fused forward and fused backward kernels (time_next_kernel)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for e in (x for row in kev for x in row):
+        e.record(stream)  # creates the CUDA events before the timed region
     barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(dev.index) as clocks:
@@ -232,8 +243,10 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
         start.record(stream)
         for s in range(args.steps):
             ev[s][0].record(stream)
+            fa.time_next_kernel(kev[s][0], kev[s][1])
             fa.forward(q, k, v, causal=w.causal, seqlens=sl, scale=w.scale, out=o, lse=lse)
             ev[s][1].record(stream)
+            fa.time_next_kernel(kev[s][2], kev[s][3])
             fa.backward(q, k, v, o, do, lse, causal=w.causal, seqlens=sl, scale=w.scale,
                         dq=dq, dk=dk, dv=dv, workspace=ws)
             ev[s][2].record(stream)
@@ -243,12 +256,15 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     elapsed_ms = start.elapsed_time(end)
     fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
     bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    fwd_kernel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in kev)
+    bwd_kernel_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in kev)
     status = fa.check_device_error(dev)
     if status != 0:
         raise RuntimeError(f"device error flag {status} after the timed region")
 
     # ---- end-to-end through the public API: pinned host inputs in, host results out
-    host_out = {n: torch.empty_like(pinned["q"]).pin_memory() for n in ("o", "dq", "dk", "dv")}
+    host_out = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory()
+                for n, t in (("o", o), ("dq", dq), ("dk", dk), ("dv", dv))}
     h2d = sum(t.numel() * t.element_size() for t in pinned.values())
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
     e2e_steps = max(1, min(args.steps, 5))
@@ -268,8 +284,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     barrier()
     e2e_ms = e0.elapsed_time(e1)
 
-    elapsed_ms, e2e_ms, fwd_ms, bwd_ms = reduce_max([elapsed_ms, e2e_ms, fwd_ms, bwd_ms], world,
-                                                    dev)
+    elapsed_ms, e2e_ms, fwd_ms, bwd_ms, fwd_kernel_ms, bwd_kernel_ms = reduce_max(
+        [elapsed_ms, e2e_ms, fwd_ms, bwd_ms, fwd_kernel_ms, bwd_kernel_ms], world, dev)
     if rank != 0:
         return None
 
@@ -279,6 +295,9 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     ms_per_step = elapsed_ms / args.steps
     bwd_tflops = bwd_flops / (bwd_ms * 1e-3) / 1e12
     fwd_tflops = fwd_flops / (fwd_ms * 1e-3) / 1e12
+    # every backward GEMM (recompute S, dP, dV, dK, dQ) runs in the fused kernel
+    bwd_kernel_tflops = bwd_flops / (bwd_kernel_ms * 1e-3) / 1e12
+    fwd_kernel_tflops = fwd_flops / (fwd_kernel_ms * 1e-3) / 1e12
     wname = args.workload
     traffic = dram_traffic("fa_bwd_kernel", wname)
     line = {
@@ -295,7 +314,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) draws rounded to bf16)",
         "pct_of_dense_bf16_peak": round(100.0 * value / world / NOMINAL_PEAK_TFLOPS, 2),
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.kv_heads, "N": w.N, "d": w.d,
                    "causal": w.causal, "padded": w.pad_range is not None,
                    "per_gpu_batch": w.B, "global_batch": w.B * world,
                    "parallelism": f"independent batches x{world}",
@@ -306,17 +325,18 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
                    "fwd_pct_of_2250": round(100 * fwd_tflops / NOMINAL_PEAK_TFLOPS, 2),
                    "bwd_pct_of_2250": round(100 * bwd_tflops / NOMINAL_PEAK_TFLOPS, 2)},
         "roofline": {
-            "kernel": "fa_bwd (preprocess + fused backward + dQ convert; the fused backward "
-                      "kernel is ~95% of the pass)",
-            "bound": "tensor", "achieved": round(bwd_tflops, 2),
+            "kernel": "fa_bwd_kernel (fused backward: all five backward GEMMs)",
+            "bound": "tensor", "achieved": round(bwd_kernel_tflops, 2),
             "peak": sustained, "unit": "TFLOP/s",
-            "frac": round(bwd_tflops / sustained, 4),
+            "frac": round(bwd_kernel_tflops / sustained, 4),
             "peak_source": f"{peak_src} bf16 sustained (MEASURED_PEAKS.json)",
+            "kernel_ms": round(bwd_kernel_ms, 4),
             "traffic": traffic,
         },
         "roofline_fwd": {
-            "kernel": "fa_fwd_kernel", "bound": "tensor", "achieved": round(fwd_tflops, 2),
-            "peak": sustained, "unit": "TFLOP/s", "frac": round(fwd_tflops / sustained, 4),
+            "kernel": "fa_fwd_kernel", "bound": "tensor", "achieved": round(fwd_kernel_tflops, 2),
+            "peak": sustained, "unit": "TFLOP/s", "frac": round(fwd_kernel_tflops / sustained, 4),
+            "kernel_ms": round(fwd_kernel_ms, 4),
             "traffic": dram_traffic("fa_fwd_kernel", wname),
         },
         "e2e": {"value": round(step_flops * e2e_steps * world / (e2e_ms * 1e-3) / 1e12, 2),
@@ -342,7 +362,9 @@ def cpu_baseline(w: workloads.Workload, inp, heads: int) -> dict:
     for flat in picks:
         b, h = divmod(flat, w.H)
         L = int(inp.seqlens[b]) if inp.seqlens is not None else w.N
-        oracle.head_bwd(inp.q[b, h], inp.k[b, h], inp.v[b, h], inp.do[b, h], w.scale, w.causal, L)
+        hk = h // (w.H // w.kv_heads)
+        oracle.head_bwd(inp.q[b, h], inp.k[b, hk], inp.v[b, hk], inp.do[b, h], w.scale, w.causal,
+                        L)
         f = 4.0 * w.N * L * w.d * (0.5 if w.causal else 1.0)
         flops += 3.5 * f
     dt = time.perf_counter() - t0
@@ -366,7 +388,9 @@ def run_reference(args, rank: int, world: int) -> dict | None:
     def one(flat):
         b, h = divmod(flat, w.H)
         L = int(inp.seqlens[b]) if inp.seqlens is not None else w.N
-        oracle.head_bwd(inp.q[b, h], inp.k[b, h], inp.v[b, h], inp.do[b, h], w.scale, w.causal, L)
+        hk = h // (w.H // w.kv_heads)
+        oracle.head_bwd(inp.q[b, h], inp.k[b, hk], inp.v[b, hk], inp.do[b, h], w.scale, w.causal,
+                        L)
 
     for i in range(args.warmup):
         one(heads[i % len(heads)])
@@ -381,11 +405,328 @@ def run_reference(args, rank: int, world: int) -> dict | None:
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(dt * 1e3 / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal},
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.kv_heads, "N": w.N, "d": w.d, "causal": w.causal},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.get_threads(),
                          "kind": "oracle",
                          "sample": f"one head of {w.B * w.H} per step, fp64 fwd+bwd"},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+# ---------------------------------------------------------------------------- further rows
+# Each row below is one more entry point of the path, measured the same way as the default
+# training step: W warm-up steps, K timed steps between events on the launching stream (plus
+# the library's events around the row's main kernel), clocks sampled meanwhile, an end-to-end
+# leg with the step's inputs copied in from pinned host memory and its result copied out, and
+# the oracle timed beside it on a bounded sample.
+import dataclasses  # noqa: E402
+from typing import Callable  # noqa: E402
+
+
+@dataclasses.dataclass
+class Row:
+    config: dict                 # workload description for the JSON line
+    metric: str
+    unit: str                    # "TFLOP/s" or "GB/s"
+    dtype: str
+    amount: float                # algorithmic FLOPs or bytes per step (whole step)
+    kernel: str                  # the main kernel the library brackets with events
+    kernel_amount: float         # algorithmic FLOPs or bytes of that kernel per step
+    bound: str                   # "tensor" or "hbm"
+    peak: float
+    peak_source: str
+    step: Callable               # step(mark): one step; mark() right before the main kernel's call
+    h2d: list                    # (device tensor, pinned host tensor) copied in per e2e step
+    d2h: list                    # (device tensor, pinned host tensor) copied out per e2e step
+    launches: int                # our kernels per step
+    cpu: Callable[[], dict]      # the oracle on a bounded sample: {"amount", "seconds", "sample"}
+    traffic_key: str | None = None
+
+
+def _pinned_pair(t: torch.Tensor):
+    return t, torch.empty(t.shape, dtype=t.dtype).pin_memory()
+
+
+def _peaks():
+    peaks, src = load_peaks()
+    bf16 = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    return bf16, hbm, src
+
+
+def row_fwd_d256(rank: int, dev) -> Row:
+    import io_aware_exact_16_b200 as fa
+    import oracle
+    w = workloads.Workload("d256 fwd non-causal B2 H16 N4096 d256", 2, 16, 4096, 256, False,
+                           1050 + 7919 * rank)
+    inp = workloads.make_inputs(w, with_grad=False)
+    q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    flops = 4.0 * w.B * w.H * w.N * w.N * w.d
+    bf16, _, src = _peaks()
+
+    def cpu():
+        heads = workloads.seeded_sample(w.seed + 5, w.B * w.H, 2)
+        t0 = time.perf_counter()
+        for flat in heads:
+            b, h = divmod(flat, w.H)
+            oracle.head_fwd(inp.q[b, h], inp.k[b, h], inp.v[b, h], w.scale, False)
+        return {"amount": flops / (w.B * w.H) * len(heads), "seconds": time.perf_counter() - t0,
+                "sample": f"fp64 C oracle forward on {len(heads)} of {w.B * w.H} heads"}
+
+    return Row(config={"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                       "causal": False, "l2": "Q,K,V,O are 67 MB each"},
+               metric="bf16 attention forward TFLOP/s at head dim 256", unit="TFLOP/s",
+               dtype="bf16", amount=flops, kernel="fa_fwd_d256_kernel", kernel_amount=flops,
+               bound="tensor", peak=bf16, peak_source=f"{src} bf16 sustained",
+               step=lambda mark: (mark(), fa.forward(q, k, v, scale=w.scale, out=o, lse=lse)),
+               h2d=[(q, inp.q.pin_memory()), (k, inp.k.pin_memory()), (v, inp.v.pin_memory())],
+               d2h=[_pinned_pair(o)], launches=1, cpu=cpu, traffic_key="fa_fwd_d256_kernel")
+
+
+def row_fwd_fp8(rank: int, dev) -> Row:
+    import io_aware_exact_16_b200 as fa
+    import oracle
+    w = workloads.Workload("fp8 fwd non-causal B4 H16 N4096 d128", 4, 16, 4096, 128, False,
+                           1060 + 7919 * rank)
+    f = workloads.make_fp8_inputs(w)
+    q, k, v = (t.to(dev) for t in (f.q, f.k, f.v))
+    qd, kd, vd = (t.to(dev) for t in (f.q_descale, f.k_descale, f.v_descale))
+    o = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    flops = 4.0 * w.B * w.H * w.N * w.N * w.d
+    bf16, _, src = _peaks()
+
+    def cpu():
+        heads = workloads.seeded_sample(w.seed + 5, w.B * w.H, 2)
+        t0 = time.perf_counter()
+        for flat in heads:
+            b, h = divmod(flat, w.H)
+            oracle.attention_fwd_fp8(f.q[b:b + 1, h:h + 1], f.k[b:b + 1, h:h + 1],
+                                     f.v[b:b + 1, h:h + 1], f.q_descale[b:b + 1, h:h + 1],
+                                     f.k_descale[b:b + 1, h:h + 1],
+                                     f.v_descale[b:b + 1, h:h + 1], w.scale, False)
+        return {"amount": flops / (w.B * w.H) * len(heads), "seconds": time.perf_counter() - t0,
+                "sample": f"fp64 oracle on the dequantised inputs, {len(heads)} of "
+                          f"{w.B * w.H} heads"}
+
+    # e4m3 tensor peak = measured bf16 peak x the nominal fp8 / bf16 ratio (4.5 / 2.25)
+    return Row(config={"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                       "causal": False, "l2": "Q,K,V 34 MB each (e4m3) + O 67 MB"},
+               metric="fp8 (e4m3) attention forward TFLOP/s", unit="TFLOP/s", dtype="e4m3",
+               amount=flops, kernel="fa_fwd_fp8_kernel", kernel_amount=flops, bound="tensor",
+               peak=2.0 * bf16, peak_source=f"{src} bf16 sustained x 2 (nominal e4m3/bf16 ratio)",
+               step=lambda mark: (mark(), fa.forward_fp8(q, k, v, qd, kd, vd, scale=w.scale,
+                                                         out=o, lse=lse)),
+               h2d=[(q, f.q.pin_memory()), (k, f.k.pin_memory()), (v, f.v.pin_memory())],
+               d2h=[_pinned_pair(o)], launches=1, cpu=cpu, traffic_key="fa_fwd_fp8_kernel")
+
+
+def row_decode(rank: int, dev) -> Row:
+    import io_aware_exact_16_b200 as fa
+    import oracle
+    B, H, H_kv, Nq, N, d = 8, 32, 8, 1, 8192, 128
+    g = torch.Generator().manual_seed(1070 + 7919 * rank)
+    q_h = torch.randn((B, H, Nq, d), generator=g).to(torch.bfloat16)
+    k_h = torch.randn((B, H_kv, N, d), generator=g).to(torch.bfloat16)
+    v_h = torch.randn((B, H_kv, N, d), generator=g).to(torch.bfloat16)
+    q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=dev)
+    splits = fa.decode_num_splits(B, H, H_kv, Nq, N, d)
+    ws = torch.empty(max(1, int(fa.decode_workspace_size(B, H, Nq, d, splits))),
+                     dtype=torch.uint8, device=dev)
+    cache_bytes = 2.0 * B * H_kv * N * d * 2
+    step_bytes = cache_bytes + 2.0 * B * H * Nq * d * 2 + 4.0 * B * H * Nq
+    _, hbm, src = _peaks()
+
+    def cpu():
+        t0 = time.perf_counter()
+        oracle.attention_decode(q_h[:1], k_h[:1], v_h[:1], d ** -0.5, False)
+        return {"amount": step_bytes / B, "seconds": time.perf_counter() - t0,
+                "sample": f"fp64 oracle decode of 1 of {B} sequences (all heads)"}
+
+    return Row(config={"workload": f"decode B{B} H{H} Hkv{H_kv} Nq{Nq} N{N} d{d}", "B": B,
+                       "H": H, "H_kv": H_kv, "Nq": Nq, "N": N, "d": d, "splits": splits,
+                       "l2": "KV cache 268 MB > L2"},
+               metric="decode attention HBM GB/s (KV-cache read)", unit="GB/s", dtype="bf16",
+               amount=step_bytes, kernel="fa_decode_kernel", kernel_amount=cache_bytes,
+               bound="hbm", peak=hbm, peak_source=f"{src} copy bandwidth",
+               step=lambda mark: (mark(), fa.decode(q, k, v, splits=splits, out=o, lse=lse,
+                                                    workspace=ws)),
+               h2d=[(q, q_h.pin_memory())], d2h=[_pinned_pair(o)],
+               launches=2 if splits > 1 else 1, cpu=cpu, traffic_key="fa_decode_kernel")
+
+
+def row_varlen(rank: int, dev) -> Row:
+    import io_aware_exact_16_b200 as fa
+    import oracle
+    w = workloads.PackedWorkload("varlen causal train B8 H16 d128 lengths U[512, 8192]", 8, 16,
+                                 16, 128, True, 1080 + 7919 * rank, len_range=(512, 8192))
+    inp = workloads.make_packed_inputs(w)
+    q, k, v, do = (t.to(dev) for t in (inp.q, inp.k, inp.v, inp.do))
+    cu = inp.cu_seqlens.to(dev)
+    lens = [int(inp.cu_seqlens[i + 1] - inp.cu_seqlens[i]) for i in range(w.B)]
+    o = torch.empty_like(q)
+    lse = torch.empty((w.H, q.shape[0]), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.bwd_workspace_size(w.B, w.H, inp.max_seqlen, w.d), dtype=torch.uint8,
+                     device=dev)
+    fwd = sum(4.0 * w.H * L * L * w.d / 2.0 for L in lens)
+    bf16, _, src = _peaks()
+
+    def step(mark):
+        fa.forward_varlen(q, k, v, cu, inp.max_seqlen, causal=True, scale=w.scale, out=o, lse=lse)
+        mark()
+        fa.backward_varlen(q, k, v, o, do, lse, cu, inp.max_seqlen, causal=True, scale=w.scale,
+                           dq=dq, dk=dk, dv=dv, workspace=ws)
+
+    def cpu():
+        b = min(range(w.B), key=lambda i: lens[i])  # the shortest sequence, one head
+        t0, t1 = int(inp.cu_seqlens[b]), int(inp.cu_seqlens[b + 1])
+        c0 = time.perf_counter()
+        oracle.head_bwd(inp.q[t0:t1, 0], inp.k[t0:t1, 0], inp.v[t0:t1, 0], inp.do[t0:t1, 0],
+                        w.scale, True)
+        L = t1 - t0
+        return {"amount": 3.5 * 4.0 * L * L * w.d / 2.0, "seconds": time.perf_counter() - c0,
+                "sample": f"fp64 C oracle fwd+bwd of one head of the shortest sequence (L={L})"}
+
+    return Row(config={"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "causal": True,
+                       "total_tokens": int(q.shape[0]), "max_seqlen": inp.max_seqlen,
+                       "l2": "Q,K,V,O,dO,dQ,dK,dV about %.0f MB each" % (q.numel() * 2 / 1e6)},
+               metric="bf16 packed variable-length attention fwd/bwd TFLOP/s", unit="TFLOP/s",
+               dtype="bf16", amount=3.5 * fwd, kernel="fa_bwd_kernel (packed)",
+               kernel_amount=2.5 * fwd, bound="tensor", peak=bf16,
+               peak_source=f"{src} bf16 sustained", step=step,
+               h2d=[(q, inp.q.pin_memory()), (k, inp.k.pin_memory()), (v, inp.v.pin_memory()),
+                    (do, inp.do.pin_memory())],
+               d2h=[_pinned_pair(t) for t in (o, dq, dk, dv)], launches=4, cpu=cpu)
+
+
+ROWS = {"fwd-d256": row_fwd_d256, "fwd-fp8": row_fwd_fp8, "decode": row_decode,
+        "varlen": row_varlen}
+
+
+def run_row(args, rank: int, world: int, local_rank: int) -> dict | None:
+    import io_aware_exact_16_b200 as fa
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    row = ROWS[args.row](rank, dev)
+    stream = torch.cuda.current_stream(dev)
+    no_mark = lambda: None  # noqa: E731
+    for _ in range(args.warmup):
+        row.step(no_mark)
+    torch.cuda.synchronize(dev)
+    if fa.check_device_error(dev) != 0:
+        raise RuntimeError("device error flag set during warm-up")
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    for e in (x for pair in kev for x in pair):
+        e.record(stream)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clocks:
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for s_ in range(args.steps):
+            row.step(lambda: fa.time_next_kernel(kev[s_][0], kev[s_][1]))
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    elapsed_ms = start.elapsed_time(end)
+    kernel_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+    if fa.check_device_error(dev) != 0:
+        raise RuntimeError("device error flag set in the timed region")
+
+    e2e_steps = max(1, min(args.steps, 10))
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for dst, src in row.h2d:
+            dst.copy_(src, non_blocking=True)
+        row.step(no_mark)
+        for src, dst in row.d2h:
+            dst.copy_(src, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    elapsed_ms, kernel_ms, e2e_ms = reduce_max([elapsed_ms, kernel_ms, e2e_ms], world, dev)
+    if rank != 0:
+        return None
+
+    scale_unit = 1e12 if row.unit == "TFLOP/s" else 1e9
+    value = row.amount * args.steps * world / (elapsed_ms * 1e-3) / scale_unit
+    achieved = row.kernel_amount / (kernel_ms * 1e-3) / scale_unit
+    traffic = dram_traffic(row.traffic_key, row.config["workload"]) if row.traffic_key else None
+    line = {
+        "metric": row.metric, "value": round(value, 2), "unit": row.unit, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(elapsed_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": row.dtype,
+        "data": "synthetic (seeded N(0,1) draws)", "row": args.row,
+        "config": dict(row.config, parallelism=f"independent batches x{world}"),
+        "roofline": {"kernel": row.kernel, "bound": row.bound, "achieved": round(achieved, 2),
+                     "peak": row.peak, "unit": row.unit, "frac": round(achieved / row.peak, 4),
+                     "peak_source": row.peak_source, "kernel_ms": round(kernel_ms, 4),
+                     "traffic": traffic},
+        "e2e": {"value": round(row.amount * e2e_steps * world / (e2e_ms * 1e-3) / scale_unit, 2),
+                "unit": row.unit,
+                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t, _ in row.h2d),
+                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t, _ in row.d2h),
+                "steps": e2e_steps},
+        "gpu_launches": row.launches * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        c = row.cpu()
+        line["cpu_baseline"] = {"value": round(c["amount"] / c["seconds"] / scale_unit, 6),
+                                "unit": row.unit, "cores": oracle.get_threads(),
+                                "kind": "oracle", "sample": f"{c['sample']} ({c['seconds']:.1f} s)"}
+    return line
+
+
+def run_row_reference(args, rank: int, world: int) -> dict | None:
+    """The oracle on the row's workload: its bounded sample (Row.cpu) once per step."""
+    if rank != 0:
+        return None
+    import oracle
+    oracle.build()
+    row = ROWS[args.row](0, torch.device("cuda", 0))
+    for _ in range(args.warmup):
+        row.cpu()
+    amount = seconds = 0.0
+    sample = ""
+    for _ in range(args.steps):
+        c = row.cpu()
+        amount += c["amount"]
+        seconds += c["seconds"]
+        sample = c["sample"]
+    scale_unit = 1e12 if row.unit == "TFLOP/s" else 1e9
+    value = amount / seconds / scale_unit
+    return {
+        "impl": "reference", "metric": row.metric, "value": round(value, 6), "unit": row.unit,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(seconds * 1e3 / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "row": args.row, "config": row.config,
+        "cpu_baseline": {"value": round(value, 6), "unit": row.unit,
+                         "cores": oracle.get_threads(), "kind": "oracle",
+                         "sample": f"{sample}, once per step"},
+        "e2e": {"value": round(value, 6), "unit": row.unit, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
 
@@ -396,7 +737,11 @@ def main() -> int:
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD,
+                    help="workload of the default training row")
+    ap.add_argument("--row", choices=["train"] + sorted(ROWS), default="train",
+                    help="train: forward + backward step (default); others: the further "
+                         "entry points, each on its own workload")
     ap.add_argument("--cpu-heads", type=int, default=12)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -415,7 +760,10 @@ def main() -> int:
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        if args.impl == "reference":
+        if args.row != "train":
+            line = (run_row_reference(args, rank, world) if args.impl == "reference"
+                    else run_row(args, rank, world, local_rank))
+        elif args.impl == "reference":
             line = run_reference(args, rank, world)
         else:
             line = run_ours(args, rank, world, local_rank)

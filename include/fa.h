@@ -128,6 +128,16 @@ FA_API fa_status fa_check_device_error(fa_stream_t stream);
 FA_API void fa_set_wait_timeout_ns(uint64_t ns);
 
 /*
+ * Measurement hook.  The next attention call made on this host thread (any fa_fwd*, fa_bwd*,
+ * fa_fwd_fp8 or fa_fwd_decode) records `start_event` on its stream immediately before its main
+ * fused kernel and `stop_event` immediately after it (the backward's preprocess and dQ
+ * convert kernels, and the decode combine kernel, fall outside), then forgets both.  The
+ * events are cudaEvent_t handles the caller created (NULL: not recorded).  This lets a caller
+ * time one kernel with CUDA events on the launching stream.
+ */
+FA_API void fa_set_kernel_timing_events(void* start_event, void* stop_event);
+
+/*
  * Grouped-query / multi-query attention (FlashAttention (DE), section on FlashAttention-2:
  * support for multi-query attention).  Same as fa_fwd / fa_bwd, except that K and V (and dK,
  * dV) have H_kv heads, [B, H_kv, N, d], with H % H_kv == 0: query head h attends with key/value

@@ -59,6 +59,8 @@ _lib.fa_bwd_workspace_size.argtypes = [_i, _i, _i, _i]
 _lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
 _lib.fa_check_device_error.argtypes = [_vp]
 _lib.fa_check_device_error.restype = _i
+_lib.fa_set_kernel_timing_events.argtypes = [_vp, _vp]
+_lib.fa_set_kernel_timing_events.restype = None
 _lib.fa_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
 _lib.fa_set_wait_timeout_ns.restype = None
 _lib.fa_status_string.argtypes = [_i]
@@ -68,7 +70,8 @@ _lib.fa_status_string.restype = ctypes.c_char_p
 EXPORTED = ("fa_fwd", "fa_bwd", "fa_fwd_gqa", "fa_bwd_gqa", "fa_fwd_varlen", "fa_bwd_varlen",
             "fa_decode_num_splits", "fa_decode_workspace_size", "fa_fwd_decode",
             "fa_fwd_fp8", "fa_bwd_workspace_size",
-            "fa_check_device_error", "fa_set_wait_timeout_ns", "fa_status_string",
+            "fa_check_device_error", "fa_set_wait_timeout_ns", "fa_set_kernel_timing_events",
+            "fa_status_string",
             "fa_bwd_noalloc")
 
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_WORKSPACE = range(6)
@@ -311,6 +314,10 @@ def decode_num_splits(B: int, H: int, H_kv: int, Nq: int, N: int, d: int) -> int
     return int(_lib.fa_decode_num_splits(B, H, H_kv, Nq, N, d))
 
 
+def decode_workspace_size(B: int, H: int, Nq: int, d: int, splits: int) -> int:
+    return int(_lib.fa_decode_workspace_size(B, H, Nq, d, splits))
+
+
 def decode(q, k_cache, v_cache, cache_lens: Optional[torch.Tensor] = None, causal: bool = False,
            scale: Optional[float] = None, splits: int = 0, out=None, lse=None,
            workspace: Optional[torch.Tensor] = None):
@@ -365,6 +372,15 @@ def check_device_error(device: Optional[torch.device] = None) -> int:
 
 def set_wait_timeout_ns(ns: int) -> None:
     _lib.fa_set_wait_timeout_ns(int(ns))
+
+
+def time_next_kernel(start: "torch.cuda.Event", stop: "torch.cuda.Event") -> None:
+    """``fa_set_kernel_timing_events``: the next call on this thread records `start` / `stop`
+    (torch CUDA events created with enable_timing=True) around its main fused kernel."""
+    for e in (start, stop):
+        if e.cuda_event == 0:  # torch creates the CUDA event lazily, on its first record
+            e.record()
+    _lib.fa_set_kernel_timing_events(start.cuda_event, stop.cuda_event)
 
 
 def raw_library() -> ctypes.CDLL:

@@ -23,6 +23,16 @@ constexpr int kMaxDevices = 64;
 
 std::atomic<uint64_t> g_timeout_ns{4000000000ull};
 
+// fa_set_kernel_timing_events: consumed by the next entry point called on this host thread.
+thread_local cudaEvent_t t_ev_start = nullptr;
+thread_local cudaEvent_t t_ev_stop = nullptr;
+
+void take_timing_events(cudaEvent_t* start, cudaEvent_t* stop) {
+    *start = t_ev_start;
+    *stop = t_ev_stop;
+    t_ev_start = t_ev_stop = nullptr;
+}
+
 struct DeviceState {
     bool probed = false;
     bool supported = false;
@@ -194,8 +204,12 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
     p.timeout_ns = g_timeout_ns.load();
+    cudaEvent_t ev0, ev1;
+    take_timing_events(&ev0, &ev1);
+    if (ev0) cudaEventRecord(ev0, stream);
     const cudaError_t e = d == 256 ? launch_fwd_d256(tq, tk, tv, p, B, stream)
                                    : launch_fwd(d, tq, tk, tv, p, B, dev->num_sms, stream);
+    if (ev1) cudaEventRecord(ev1, stream);
     if (e != cudaSuccess) return FA_ERR_CUDA;
     return FA_OK;
 }
@@ -247,6 +261,11 @@ const char* fa_status_string(fa_status s) {
         case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: workspace missing, misaligned or too small";
     }
     return "unknown fa_status";
+}
+
+void fa_set_kernel_timing_events(void* start_event, void* stop_event) {
+    t_ev_start = static_cast<cudaEvent_t>(start_event);
+    t_ev_stop = static_cast<cudaEvent_t>(stop_event);
 }
 
 void fa_set_wait_timeout_ns(uint64_t ns) {
@@ -343,7 +362,9 @@ static fa_status bwd_impl(const void* q, const void* k, const void* v, const voi
     if (!user_map(&tq, q, d, B, H, N, T, packed) || !user_map(&tk, k, d, B, H_kv, N, T, packed) ||
         !user_map(&tv, v, d, B, H_kv, N, T, packed) || !user_map(&tdo, dO, d, B, H, N, T, packed))
         return FA_ERR_CUDA;
-    if (launch_bwd(d, tq, tk, tv, tdo, p, stream) != cudaSuccess) return FA_ERR_CUDA;
+    cudaEvent_t ev0, ev1;
+    take_timing_events(&ev0, &ev1);
+    if (launch_bwd(d, tq, tk, tv, tdo, p, stream, ev0, ev1) != cudaSuccess) return FA_ERR_CUDA;
     return FA_OK;
 }
 
@@ -409,8 +430,13 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, const float* q
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
     p.timeout_ns = g_timeout_ns.load();
-    if (launch_fwd_fp8(tq, tk, tv, p, B, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-        return FA_ERR_CUDA;
+    cudaEvent_t ev0, ev1;
+    take_timing_events(&ev0, &ev1);
+    const cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
+    if (ev0) cudaEventRecord(ev0, st_);
+    const cudaError_t e = launch_fwd_fp8(tq, tk, tv, p, B, st_);
+    if (ev1) cudaEventRecord(ev1, st_);
+    if (e != cudaSuccess) return FA_ERR_CUDA;
     return FA_OK;
 }
 
@@ -490,7 +516,10 @@ fa_status fa_fwd_decode(const void* q, const void* k_cache, const void* v_cache,
         !make_bf16_map(&tk, k_cache, d, N, B * H_kv, 128) ||
         !make_bf16_map(&tv, v_cache, d, N, B * H_kv, 128))
         return FA_ERR_CUDA;
-    if (launch_decode(d, tq, tk, tv, p, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    cudaEvent_t ev0, ev1;
+    take_timing_events(&ev0, &ev1);
+    if (launch_decode(d, tq, tk, tv, p, reinterpret_cast<cudaStream_t>(stream), ev0, ev1) !=
+        cudaSuccess)
         return FA_ERR_CUDA;
     return FA_OK;
 }

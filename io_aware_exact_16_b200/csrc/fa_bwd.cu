@@ -750,7 +750,8 @@ __global__ void __launch_bounds__(512, 1)
 
 template <int D, bool PACKED>
 cudaError_t launch_bwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                         const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream) {
+                         const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream,
+                         cudaEvent_t ev_start, cudaEvent_t ev_stop) {
     using C = BwdCfg<D>;
     static bool configured = false;
     if (!configured) {
@@ -765,7 +766,9 @@ cudaError_t launch_bwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
     const int BHkv = p.B * p.H_kv;
     const dim3 chunks(p.N_pad / 128, BH);
     fa_bwd_pre_kernel<D><<<chunks, 256, 0, stream>>>(p);
+    if (ev_start) cudaEventRecord(ev_start, stream);
     fa_bwd_kernel<D, PACKED><<<BHkv * n_kv, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
+    if (ev_stop) cudaEventRecord(ev_stop, stream);
     fa_bwd_dq_kernel<D><<<chunks, 256, 0, stream>>>(p);
     return cudaGetLastError();
 }
@@ -773,13 +776,14 @@ cudaError_t launch_bwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 }  // namespace
 
 cudaError_t launch_bwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream) {
+                       const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream,
+                       cudaEvent_t ev_start, cudaEvent_t ev_stop) {
     const bool packed = p.cu_seqlens != nullptr;
     if (d == 64)
-        return packed ? launch_bwd_d<64, true>(tq, tk, tv, tdo, p, stream)
-                      : launch_bwd_d<64, false>(tq, tk, tv, tdo, p, stream);
-    return packed ? launch_bwd_d<128, true>(tq, tk, tv, tdo, p, stream)
-                  : launch_bwd_d<128, false>(tq, tk, tv, tdo, p, stream);
+        return packed ? launch_bwd_d<64, true>(tq, tk, tv, tdo, p, stream, ev_start, ev_stop)
+                      : launch_bwd_d<64, false>(tq, tk, tv, tdo, p, stream, ev_start, ev_stop);
+    return packed ? launch_bwd_d<128, true>(tq, tk, tv, tdo, p, stream, ev_start, ev_stop)
+                  : launch_bwd_d<128, false>(tq, tk, tv, tdo, p, stream, ev_start, ev_stop);
 }
 
 }  // namespace fa

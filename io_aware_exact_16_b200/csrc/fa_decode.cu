@@ -465,7 +465,8 @@ __global__ void __launch_bounds__(256) fa_decode_combine_kernel(const DecodePara
 
 template <int D>
 cudaError_t launch_decode_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const DecodeParams& p, cudaStream_t stream) {
+                            const DecodeParams& p, cudaStream_t stream, cudaEvent_t ev_start,
+                            cudaEvent_t ev_stop) {
     using C = DecCfg<D>;
     static bool configured = false;  // attribute set once per process (idempotent if raced)
     if (!configured) {
@@ -476,7 +477,9 @@ cudaError_t launch_decode_d(const CUtensorMap& tq, const CUtensorMap& tk, const 
         configured = true;
     }
     const dim3 grid(p.splits, p.H_kv * p.n_mtiles, p.B);
+    if (ev_start) cudaEventRecord(ev_start, stream);
     fa_decode_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    if (ev_stop) cudaEventRecord(ev_stop, stream);
     if (p.splits > 1) {
         const size_t rows = (size_t)p.B * p.H * p.Nq;
         fa_decode_combine_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(p);
@@ -487,10 +490,11 @@ cudaError_t launch_decode_d(const CUtensorMap& tq, const CUtensorMap& tk, const 
 }  // namespace
 
 cudaError_t launch_decode(int d, const CUtensorMap& tq, const CUtensorMap& tk,
-                          const CUtensorMap& tv, const DecodeParams& p, cudaStream_t stream) {
-    if (d == 64) return launch_decode_d<64>(tq, tk, tv, p, stream);
-    if (d == 256) return launch_decode_d<256>(tq, tk, tv, p, stream);
-    return launch_decode_d<128>(tq, tk, tv, p, stream);
+                          const CUtensorMap& tv, const DecodeParams& p, cudaStream_t stream,
+                          cudaEvent_t ev_start, cudaEvent_t ev_stop) {
+    if (d == 64) return launch_decode_d<64>(tq, tk, tv, p, stream, ev_start, ev_stop);
+    if (d == 256) return launch_decode_d<256>(tq, tk, tv, p, stream, ev_start, ev_stop);
+    return launch_decode_d<128>(tq, tk, tv, p, stream, ev_start, ev_stop);
 }
 
 }  // namespace fa

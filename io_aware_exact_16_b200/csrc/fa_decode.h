@@ -26,7 +26,9 @@ struct DecodeParams {
 };
 
 // Query tile map: q [B, H, Nq, d] seen as (d, G*Nq, B*H_kv); cache maps as make_bf16_map.
+// ev_start / ev_stop (optional) bracket the split kernel on `stream` (not the combine).
 cudaError_t launch_decode(int d, const CUtensorMap& tq, const CUtensorMap& tk,
-                          const CUtensorMap& tv, const DecodeParams& p, cudaStream_t stream);
+                          const CUtensorMap& tv, const DecodeParams& p, cudaStream_t stream,
+                          cudaEvent_t ev_start = nullptr, cudaEvent_t ev_stop = nullptr);
 
 }  // namespace fa

@@ -120,7 +120,10 @@ bool make_bf16_map_packed(CUtensorMap* map, const void* base, int d, int Hx, int
 cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const FwdParams& p, int B, int num_sms, cudaStream_t stream);
 
+// ev_start / ev_stop (optional) are recorded on `stream` right before and after the fused
+// backward kernel (between the preprocess and the dQ convert kernels).
 cudaError_t launch_bwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream);
+                       const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream,
+                       cudaEvent_t ev_start = nullptr, cudaEvent_t ev_stop = nullptr);
 
 }  // namespace fa
