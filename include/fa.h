@@ -201,11 +201,11 @@ FA_API fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, cons
  *                  j <= L_b - Nq + i (aligned to the end of the cache); a query that sees no
  *                  key gets O = 0 and lse = -inf.
  *   splits         key ranges per (sequence, cache head) computed by separate CTAs and merged
- *                  by their log-sum-exp; 0 = fa_decode_num_splits(...).  The value is capped at
- *                  the number of 128-key blocks of N.
+ *                  by their log-sum-exp; 0 = fa_decode_num_splits(...).  Ranges hold whole key
+ *                  blocks (64 keys for d <= 128, 128 for d = 256), so the count used may be
+ *                  lower than the one requested.
  *   workspace      device, 16-byte aligned, >= fa_decode_workspace_size(B, H, Nq, d, splits)
- *                  bytes when splits > 1 (pass the splits the call will use); may be NULL
- *                  when splits == 1.
+ *                  bytes for the requested splits when they exceed 1; may be NULL otherwise.
  * d in {64, 128, 256}.  The result is exact for every `splits` (up to rounding: different
  * splits round differently; the same splits give identical bits).
  */

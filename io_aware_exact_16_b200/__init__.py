@@ -344,11 +344,8 @@ def decode(q, k_cache, v_cache, cache_lens: Optional[torch.Tensor] = None, causa
         raise ValueError("lse must be a contiguous float32 tensor [B, H, Nq]")
     if splits == 0:
         splits = decode_num_splits(B, H, H_kv, Nq, N, d)
-    nblk = (N + 127) // 128
-    splits = max(1, min(int(splits), nblk))
-    bps = (nblk + splits - 1) // splits
-    splits = (nblk + bps - 1) // bps
-    need = int(_lib.fa_decode_workspace_size(B, H, Nq, d, splits))
+    splits = max(1, int(splits))
+    need = int(_lib.fa_decode_workspace_size(B, H, Nq, d, splits))  # enough for any count used
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_ptr = workspace.data_ptr() if workspace is not None else None

@@ -214,17 +214,18 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
     return FA_OK;
 }
 
-// Split-KV decode: the number of key ranges that minimises (waves of CTAs) x (128-key blocks
-// per CTA + 1 for its fixed cost), preferring fewer ranges on ties.
-int decode_splits(int B, int H_kv, int n_mt, int N, int num_sms) {
-    const int nblk = (N + 127) / 128;
+// Split-KV decode: the number of key ranges that minimises (waves of CTAs) x (key blocks per
+// CTA + 1 for its fixed cost), preferring fewer ranges on ties.  `bk` keys per block, `slots`
+// CTAs resident per wave.
+int decode_splits(int B, int H_kv, int n_mt, int N, int bk, int slots) {
+    const int nblk = (N + bk - 1) / bk;
     const long long base = (long long)B * H_kv * n_mt;
     int best = 1;
     long long best_cost = -1;
     for (int s = 1; s <= nblk && s <= 256; ++s) {
         const int bps = (nblk + s - 1) / s;
         if ((nblk + bps - 1) / bps != s) continue;  // same ranges as a smaller s
-        const long long waves = (base * s + num_sms - 1) / num_sms;
+        const long long waves = (base * s + slots - 1) / slots;
         const long long cost = waves * (bps + 1);
         if (best_cost < 0 || cost < best_cost) {
             best_cost = cost;
@@ -449,7 +450,7 @@ int fa_decode_num_splits(int B, int H, int H_kv, int Nq, int N, int d) {
             sms = v;
     }
     const int n_mt = ((H / H_kv) * Nq + 127) / 128;
-    return decode_splits(B, H_kv, n_mt, N, sms);
+    return decode_splits(B, H_kv, n_mt, N, decode_block_keys(d), sms * decode_ctas_per_sm(d));
 }
 
 size_t fa_decode_workspace_size(int B, int H, int Nq, int d, int splits) {
@@ -476,8 +477,10 @@ fa_status fa_fwd_decode(const void* q, const void* k_cache, const void* v_cache,
 
     const int G = H / H_kv;
     const int n_mt = (G * Nq + 127) / 128;
-    const int nblk = (N + 127) / 128;
-    if (splits == 0) splits = decode_splits(B, H_kv, n_mt, N, dev->num_sms);
+    const int bk = decode_block_keys(d);
+    const int nblk = (N + bk - 1) / bk;
+    if (splits == 0)
+        splits = decode_splits(B, H_kv, n_mt, N, bk, dev->num_sms * decode_ctas_per_sm(d));
     if (splits > nblk) splits = nblk;
     const int bps = (nblk + splits - 1) / splits;
     splits = (nblk + bps - 1) / bps;  // ranges that actually hold keys
@@ -513,8 +516,8 @@ fa_status fa_fwd_decode(const void* q, const void* k_cache, const void* v_cache,
 
     CUtensorMap tq, tk, tv;
     if (!make_bf16_map(&tq, q, d, G * Nq, B * H_kv, 128) ||
-        !make_bf16_map(&tk, k_cache, d, N, B * H_kv, 128) ||
-        !make_bf16_map(&tv, v_cache, d, N, B * H_kv, 128))
+        !make_bf16_map(&tk, k_cache, d, N, B * H_kv, bk) ||
+        !make_bf16_map(&tv, v_cache, d, N, B * H_kv, bk))
         return FA_ERR_CUDA;
     cudaEvent_t ev0, ev1;
     take_timing_events(&ev0, &ev1);

@@ -16,7 +16,7 @@
 // Decode is bound by reading the cache (each key/value row is read once, used by G * Nq query
 // rows), so the CTA keeps a deep ring of 16 KB K/V chunks in flight and double-buffers the
 // score block in tensor memory (S(j+1) is computed while the softmax works on S(j)).
-//   tensor memory:  S_a [0,128)  S_b [128,256)  O [256, 256 + d)
+//   tensor memory:  S_a [0,BN)  S_b [BN,2BN)  O [2BN, 2BN + d)   (BN keys per block)
 //   MMA order:      S(0) S(1) | PV(0) S(2) | PV(1) S(3) | ...
 // Warp roles (192 threads): warps 0-3 softmax (thread r owns tile row r = TMEM lane r), warp 4
 // MMA issue + TMEM allocation, warp 5 TMA.
@@ -34,25 +34,33 @@ namespace {
 
 using namespace sm100;
 
+// BN = 64 (d <= 128): 256 tensor-memory columns and ~105 KB of shared memory per CTA, so two
+// CTAs share an SM and their serial per-block chains (S -> softmax -> P V) overlap;
+// BN = 128 (d = 256): O alone needs 256 columns, one CTA per SM.
 template <int D>
 struct DecCfg {
     static constexpr int BM = 128;                   // query rows per tile
-    static constexpr int BN = 128;                   // keys per block
+    static constexpr int BN = (D == 256) ? 128 : 64; // keys per block
+    static constexpr int CTAS_PER_SM = (D == 256) ? 1 : 2;
     static constexpr int KCH = D / 64;               // 64-column chunks per row
-    static constexpr int CHUNK_BYTES = 128 * 128;    // one chunk: 128 rows x 128 bytes
-    static constexpr int NSLOT = (D == 256) ? 10 : 12;
+    static constexpr int Q_CHUNK_BYTES = BM * 128;   // a Q chunk: 128 rows x 128 bytes
+    static constexpr int CHUNK_BYTES = BN * 128;     // a K/V chunk: BN rows x 128 bytes
+    static constexpr int NSLOT = (D == 256) ? 10 : 9;
     static constexpr int SMEM_Q = 0;
-    static constexpr int SMEM_RING = SMEM_Q + KCH * CHUNK_BYTES;
+    static constexpr int SMEM_RING = SMEM_Q + KCH * Q_CHUNK_BYTES;
     static constexpr int SMEM_BAR = SMEM_RING + NSLOT * CHUNK_BYTES;
     // q, full[NSLOT], empty[NSLOT], sfull[2], pfull[2], ofull, done
     static constexpr int NUM_BARS = 1 + 2 * NSLOT + 2 + 2 + 1 + 1;
     static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;  // + alignment slack
     static constexpr int THREADS = 192;
-    static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr uint32_t TM_O = 256;
-    __device__ static constexpr uint32_t tm_s(int buf) { return buf ? 128u : 0u; }
+    static constexpr uint32_t TM_O = 2 * BN;         // after the two score buffers
+    static constexpr uint32_t TMEM_COLS = (TM_O + D <= 256) ? 256 : 512;
+    __device__ static constexpr uint32_t tm_s(int buf) { return buf ? (uint32_t)BN : 0u; }
     static_assert(SMEM_BYTES <= 232448, "shared memory over the sm_100 per-CTA limit");
+    static_assert(CTAS_PER_SM == 1 || (SMEM_BYTES + 1024) * 2 <= 233472,
+                  "two CTAs must fit in one SM's shared memory");
+    static_assert(TM_O + D <= TMEM_COLS && TMEM_COLS * CTAS_PER_SM <= 512, "tensor memory");
 };
 
 __device__ __forceinline__ void record_error(int* err, int code) {
@@ -60,7 +68,7 @@ __device__ __forceinline__ void record_error(int* err, int code) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, DecCfg<D>::CTAS_PER_SM)
     fa_decode_kernel(const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
@@ -138,9 +146,9 @@ __global__ void __launch_bounds__(192, 1)
             prefetch_tensormap(&tmQ);
             prefetch_tensormap(&tmK);
             prefetch_tensormap(&tmV);
-            mbar_arrive_expect_tx(bar_q, C::KCH * C::CHUNK_BYTES);
+            mbar_arrive_expect_tx(bar_q, C::KCH * C::Q_CHUNK_BYTES);
             for (int c = 0; c < C::KCH; ++c)
-                tma_load_3d(smem + C::SMEM_Q + c * C::CHUNK_BYTES, &tmQ, bar_q, c * 64,
+                tma_load_3d(smem + C::SMEM_Q + c * C::Q_CHUNK_BYTES, &tmQ, bar_q, c * 64,
                             mt * C::BM, bhk);
             int u = 0;  // chunks issued into the ring
             bool ok = true;
@@ -188,7 +196,7 @@ __global__ void __launch_bounds__(192, 1)
                         return false;
                     tc_fence_after();
                     const uint32_t ka = sR + s * C::CHUNK_BYTES;
-                    const uint32_t qa = sQ + c * C::CHUNK_BYTES;
+                    const uint32_t qa = sQ + c * C::Q_CHUNK_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_ss(tmem + C::tm_s(buf), sdesc_sw128(qa + kk * 32, 16, 1024),
@@ -476,7 +484,7 @@ cudaError_t launch_decode_d(const CUtensorMap& tq, const CUtensorMap& tk, const 
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    const dim3 grid(p.splits, p.H_kv * p.n_mtiles, p.B);
+    const dim3 grid(p.splits, p.H_kv * p.n_mtiles, p.B);  // splits in units of C::BN blocks
     if (ev_start) cudaEventRecord(ev_start, stream);
     fa_decode_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
     if (ev_stop) cudaEventRecord(ev_stop, stream);
@@ -488,6 +496,11 @@ cudaError_t launch_decode_d(const CUtensorMap& tq, const CUtensorMap& tk, const 
 }
 
 }  // namespace
+
+int decode_block_keys(int d) { return d == 64 ? DecCfg<64>::BN : d == 256 ? DecCfg<256>::BN : DecCfg<128>::BN; }
+int decode_ctas_per_sm(int d) {
+    return d == 64 ? DecCfg<64>::CTAS_PER_SM : d == 256 ? DecCfg<256>::CTAS_PER_SM : DecCfg<128>::CTAS_PER_SM;
+}
 
 cudaError_t launch_decode(int d, const CUtensorMap& tq, const CUtensorMap& tk,
                           const CUtensorMap& tv, const DecodeParams& p, cudaStream_t stream,

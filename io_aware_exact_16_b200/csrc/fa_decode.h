@@ -19,13 +19,18 @@ struct DecodeParams {
     int N;                  // cache rows per head (capacity)
     int n_mtiles;           // ceil(G * Nq / 128)
     int splits;             // key ranges per (b, cache head)
-    int blocks_per_split;   // 128-key blocks per range
+    int blocks_per_split;   // key blocks (decode_block_keys(d) keys each) per range
     float scale_log2;       // scale * log2(e)
     int causal;
     uint64_t timeout_ns;
 };
 
 // Query tile map: q [B, H, Nq, d] seen as (d, G*Nq, B*H_kv); cache maps as make_bf16_map.
+// Keys per block of the decode kernel for head dim d (the unit of blocks_per_split and of the
+// K/V tensor maps' box rows) and how many of its CTAs share one SM.
+int decode_block_keys(int d);
+int decode_ctas_per_sm(int d);
+
 // ev_start / ev_stop (optional) bracket the split kernel on `stream` (not the combine).
 cudaError_t launch_decode(int d, const CUtensorMap& tq, const CUtensorMap& tk,
                           const CUtensorMap& tv, const DecodeParams& p, cudaStream_t stream,
