@@ -480,6 +480,7 @@ __global__ void __launch_bounds__(512, 1)
         const uint64_t dV_k = sdesc_sw128(smem_u32(smem + C::SMEM_V), 16, 1024);
         const uint64_t dK_mn = sdesc_sw128(smem_u32(smem + C::SMEM_K), C::CHUNK_BYTES, 1024);
         const uint64_t dDS_mn = sdesc_sw128(smem_u32(smem + C::SMEM_DS), C::CHUNK_BYTES, 1024);
+        const uint64_t dDS_k = sdesc_sw128(smem_u32(smem + C::SMEM_DS), 16, 1024);
         // Q / dO stage st sits st * Q_TILE_BYTES after stage 0.
         const uint64_t dQ_k0 = sdesc_sw128(smem_u32(smem + C::SMEM_Q), 16, 1024);
         const uint64_t dDO_k0 = sdesc_sw128(smem_u32(smem + C::SMEM_DO), 16, 1024);
@@ -532,14 +533,16 @@ __global__ void __launch_bounds__(512, 1)
                 tc_fence_after();
                 issue_S(it + 1);
             }
-            // dK += dS^T Q, same shapes as dV.
             if (!(ok = mbar_wait(bar_dsfull, it & 1, p.timeout_ns, abort_flag))) break;
             tc_fence_after();
+            if constexpr (D == 128) {
+                // dK += dS^T Q, same shapes as dV (A = dS^T in tensor memory).
 #pragma unroll
-            for (int kk = 0; kk < C::BM / 16; ++kk)
-                mma_ts(tmem + C::TM_DK, tmem + C::TM_B + kk * 8, dQ_mn + mnmaj(kk), idKV,
-                       (it > 0 || kk > 0) ? 1u : 0u);
-            tc_commit(&bar_qempty[s]);
+                for (int kk = 0; kk < C::BM / 16; ++kk)
+                    mma_ts(tmem + C::TM_DK, tmem + C::TM_B + kk * 8, dQ_mn + mnmaj(kk), idKV,
+                           (it > 0 || kk > 0) ? 1u : 0u);
+                tc_commit(&bar_qempty[s]);
+            }
             // The dQ block into B; K steps of 16 keys = 2048 bytes of both tiles, both
             // operands MN-major.
             if constexpr (D == 128) {
@@ -556,6 +559,16 @@ __global__ void __launch_bounds__(512, 1)
                            kk > 0 ? 1u : 0u);
             }
             tc_commit(bar_dqfull);
+            if constexpr (D == 64) {
+                // d = 64: dK after dQ, so the drain starts earlier; A = dS^T read from its
+                // shared-memory tile (K-major: key rows, query columns), since dQ has just
+                // overwritten tensor-memory B.  Measured faster at d = 64, slower at d = 128.
+#pragma unroll
+                for (int kk = 0; kk < C::BM / 16; ++kk)
+                    mma_ss(tmem + C::TM_DK, dDS_k + kmaj(kk), dQ_mn + mnmaj(kk), idKV,
+                           (it > 0 || kk > 0) ? 1u : 0u);
+                tc_commit(&bar_qempty[s]);
+            }
             // dP^T(it+1) into B once the drain has copied the dQ block out.
             if (it + 1 < n_it) {
                 if (!(ok = mbar_wait(bar_dqempty, it & 1, p.timeout_ns, abort_flag))) break;
@@ -692,7 +705,8 @@ __global__ void __launch_bounds__(512, 1)
             if (it + 1 < n_it) store_vectors(it + 1);
             named_barrier(1, 256);  // every dP^T column read before dS^T overwrites columns
             if (ok) {
-                tmem_st32(tmem + lane_base + C::TM_B + 32 * h, dw);
+                // d = 128: dK reads dS^T from tensor memory; d = 64 reads the shared tile below.
+                if constexpr (D == 128) tmem_st32(tmem + lane_base + C::TM_B + 32 * h, dw);
                 // dS^T row r, queries [64h, 64h+64) = one 128-byte row of query chunk h; 16-byte
                 // unit u sits at position u ^ (r % 8) (the 128-byte swizzle the MMA reads).
 #pragma unroll
