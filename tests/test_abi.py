@@ -96,3 +96,55 @@ def test_python_binding_checks_shapes_before_calling():
     kb = torch.zeros((1, 1, 9, 64), dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         fa.forward(qb, kb, qb)
+
+
+def test_gqa_and_varlen_reject_bad_arguments_without_a_device():
+    lib = fa.raw_library()
+    f = ctypes.c_float(0.125)
+    # H_kv must divide H and lie in [1, H]
+    assert lib.fa_fwd_gqa(16, 16, 16, 16, 16, 1, 4, 3, 8, 64, f, 0, None, None) == \
+        fa.FA_ERR_INVALID_ARG
+    assert lib.fa_fwd_gqa(16, 16, 16, 16, 16, 1, 4, 8, 8, 64, f, 0, None, None) == \
+        fa.FA_ERR_INVALID_ARG
+    # packed: offsets required, total >= 1, 4-byte aligned offsets
+    assert lib.fa_fwd_varlen(16, 16, 16, 16, 16, None, 2, 8, 16, 4, 4, 64, f, 0, None) == \
+        fa.FA_ERR_INVALID_ARG
+    assert lib.fa_fwd_varlen(16, 16, 16, 16, 16, 16, 2, 8, 0, 4, 4, 64, f, 0, None) == \
+        fa.FA_ERR_INVALID_ARG
+    assert lib.fa_fwd_varlen(16, 16, 16, 16, 16, 18, 2, 8, 16, 4, 4, 64, f, 0, None) == \
+        fa.FA_ERR_INVALID_ARG
+    assert lib.fa_bwd_varlen(16, 16, 16, 16, 16, 16, 16, 16, 16, 16, 2, 8, 16, 4, 4, 256, f, 0,
+                             16, 1 << 20, None) == fa.FA_ERR_UNSUPPORTED
+
+
+def test_fp8_and_decode_reject_bad_arguments_without_a_device():
+    lib = fa.raw_library()
+    f = ctypes.c_float(0.125)
+    fp8 = lambda d=128, H_kv=2, qd=None: lib.fa_fwd_fp8(  # noqa: E731
+        16, 16, 16, qd, None, None, 16, 16, 1, 4, H_kv, 64, d, f, 0, None, None)
+    assert fp8(d=64) == fa.FA_ERR_UNSUPPORTED
+    assert fp8(H_kv=3) == fa.FA_ERR_INVALID_ARG
+    assert fp8(qd=18) == fa.FA_ERR_INVALID_ARG  # descale factors must be 4-byte aligned
+    dec = lambda H=8, H_kv=2, Nq=1, N=100, d=128, splits=0, ws=None, wsb=0: lib.fa_fwd_decode(  # noqa: E731
+        16, 16, 16, 16, 16, None, 2, H, H_kv, Nq, N, d, f, 0, splits, ws, wsb, None)
+    assert dec(H_kv=3) == fa.FA_ERR_INVALID_ARG
+    assert dec(d=96) == fa.FA_ERR_UNSUPPORTED
+    assert dec(Nq=0) == fa.FA_ERR_INVALID_ARG
+    assert dec(splits=-1) == fa.FA_ERR_INVALID_ARG
+
+
+def test_decode_split_heuristic_and_workspace_size():
+    """Host logic only: the automatic split count stays within [1, key blocks] and grows when
+    the (sequence, cache head) pairs alone cannot fill the device; the workspace holds fp32
+    O and lse partials for every split (none for one split)."""
+    for (B, H, H_kv, Nq, N, d) in ((8, 32, 8, 1, 8192, 128), (1, 32, 8, 1, 131072, 128),
+                                   (64, 32, 8, 1, 2048, 64), (1, 4, 4, 1, 100, 256)):
+        s = fa.decode_num_splits(B, H, H_kv, Nq, N, d)
+        bk = 128 if d == 256 else 64
+        assert 1 <= s <= (N + bk - 1) // bk
+    assert fa.decode_num_splits(1, 32, 8, 1, 131072, 128) > fa.decode_num_splits(64, 32, 8, 1, 131072, 128)
+    assert fa.decode_workspace_size(2, 4, 3, 128, 1) == 0
+    rows = 2 * 4 * 3
+    o_bytes = (5 * rows * 128 * 4 + 255) // 256 * 256
+    assert fa.decode_workspace_size(2, 4, 3, 128, 5) == o_bytes + 5 * rows * 4
+    assert fa.decode_num_splits(1, 4, 3, 1, 100, 128) == 0  # H_kv must divide H
