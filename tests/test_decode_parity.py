@@ -39,6 +39,12 @@ CASES = [
     (1, 64, 1, 4, 1024, 64, False, None, 0),         # 256 query rows: two row tiles
     (2, 8, 2, 1, 8192, 128, False, [8192, 4097], 16),
     (1, 8, 8, 2, 4096, 256, True, None, 0),
+    # the work split: many short sequences per CTA, two query tiles cut between CTAs, more
+    # CTAs than key blocks
+    (40, 4, 2, 2, 256, 64, True, [1 + (37 * i) % 256 for i in range(40)], 3),
+    (2, 64, 2, 8, 640, 128, False, None, 5),
+    (3, 8, 1, 1, 100, 64, False, [100, 37, 64], 0),
+    (2, 8, 2, 1, 700, 128, True, [700, 333], 40),
 ]
 
 
