@@ -36,6 +36,11 @@
 #ifndef FA_FWD_EXP2_FMA_OF_4
 #define FA_FWD_EXP2_FMA_OF_4 0
 #endif
+// The softmax releases each block's P to the MMA thread in this many parts of BN / parts keys,
+// so that the P V MMAs of the first parts run while it computes the later ones.
+#ifndef FA_FWD_P_PARTS
+#define FA_FWD_P_PARTS 2
+#endif
 
 namespace fa {
 namespace {
@@ -57,7 +62,9 @@ struct FwdCfg {
     static constexpr int SMEM_K = SMEM_Q + TILES * Q_TILE_BYTES;
     static constexpr int SMEM_V = SMEM_K + STAGES * KV_TILE_BYTES;
     static constexpr int SMEM_BAR = SMEM_V + STAGES * KV_TILE_BYTES;
-    static constexpr int NUM_BARS = 1 + 4 * STAGES + 2 + 2 + 2 + 1;
+    static constexpr int P_PARTS = FA_FWD_P_PARTS;  // P released in parts of BN / P_PARTS keys
+    static_assert(P_PARTS == 2 || P_PARTS == 4, "P is released in halves or quarters");
+    static constexpr int NUM_BARS = 1 + 4 * STAGES + 2 + 2 + 2 + 2 * (P_PARTS - 1) + 1;
     static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;  // + alignment slack
     static constexpr int THREADS = 384;
@@ -118,7 +125,8 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t* bar_sfull = bar_vempty + C::STAGES;  // [2]
     uint64_t* bar_pfull = bar_sfull + 2;            // [2]
     uint64_t* bar_ofull = bar_pfull + 2;            // [2]
-    uint64_t* bar_done = bar_ofull + 2;             // every MMA of this CTA finished
+    uint64_t* bar_ppart = bar_ofull + 2;            // [2][P_PARTS-1] P of all but the last part
+    uint64_t* bar_done = bar_ppart + 2 * (C::P_PARTS - 1);  // every MMA of this CTA finished
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SMEM_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::SMEM_MISC + 4);
 
@@ -134,6 +142,7 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(&bar_sfull[t], 1);
             mbar_init(&bar_pfull[t], C::BM);
             mbar_init(&bar_ofull[t], 1);
+            for (int q = 0; q + 1 < C::P_PARTS; ++q) mbar_init(&bar_ppart[t * (C::P_PARTS - 1) + q], C::BM);
         }
         mbar_init(bar_done, 1);
         *abort_flag = 0;
@@ -212,17 +221,32 @@ __global__ void __launch_bounds__(384, 1)
                            sdesc_sw128(ka + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
                 }
             };
-            // O_t += P_t V: P from tensor memory (2 bf16 per column, 8 columns per K step of
-            // 16 keys), V MN-major in shared memory (16 key rows = 2048 bytes per K step; the
-            // two 64-column chunks of d are CHUNK_BYTES apart).
-            auto issue_PV = [&](int t, int s, bool accumulate) {
+            // O_t += P_t V over the keys of part `part` (BN / P_PARTS keys): P from tensor memory
+            // (2 bf16 per column, 8 columns per K step of 16 keys), V MN-major in shared memory
+            // (16 key rows = 2048 bytes per K step; the two 64-column chunks of d are
+            // CHUNK_BYTES apart).  The softmax releases P part by part, so the first parts'
+            // MMAs run while it computes the later parts' exponentials.
+            constexpr int KK_PART = C::BN / 16 / C::P_PARTS;  // K steps per part
+            auto issue_PV = [&](int t, int s, bool accumulate, int part) {
                 const uint32_t va = sV + s * C::KV_TILE_BYTES;
 #pragma unroll
-                for (int kk = 0; kk < C::BN / 16; ++kk) {
+                for (int kk = part * KK_PART; kk < (part + 1) * KK_PART; ++kk) {
                     mma_ts(tmem + C::tm_o(t), tmem + C::tm_s(t) + kk * 8,
                            sdesc_sw128(va + kk * 2048, C::CHUNK_BYTES, 1024), idPV,
                            (accumulate || kk > 0) ? 1u : 0u);
                 }
+            };
+            auto wait_issue_PV = [&](int t, int s, int j) {
+#pragma unroll
+                for (int part = 0; part < C::P_PARTS; ++part) {
+                    uint64_t* bar = part + 1 < C::P_PARTS
+                                        ? &bar_ppart[t * (C::P_PARTS - 1) + part]
+                                        : &bar_pfull[t];
+                    if (!mbar_wait(bar, j & 1, p.timeout_ns, abort_flag)) return false;
+                    tc_fence_after();
+                    issue_PV(t, s, j > 0 || part > 0, part);
+                }
+                return true;
             };
 
             bool ok = mbar_wait(bar_q, 0, p.timeout_ns, abort_flag);
@@ -243,9 +267,7 @@ __global__ void __launch_bounds__(384, 1)
                 const uint32_t phn = (jn / C::STAGES) & 1;
                 if (!(ok = mbar_wait(&bar_vfull[s], ph, p.timeout_ns, abort_flag))) break;
                 if (j < n0) {
-                    if (!(ok = mbar_wait(&bar_pfull[0], j & 1, p.timeout_ns, abort_flag))) break;
-                    tc_fence_after();
-                    issue_PV(0, s, j > 0);
+                    if (!(ok = wait_issue_PV(0, s, j))) break;
                     tc_commit(&bar_ofull[0]);
                 }
                 if (jn < n1) {
@@ -256,9 +278,7 @@ __global__ void __launch_bounds__(384, 1)
                         tc_commit(&bar_sfull[0]);
                     }
                 }
-                if (!(ok = mbar_wait(&bar_pfull[1], j & 1, p.timeout_ns, abort_flag))) break;
-                tc_fence_after();
-                issue_PV(1, s, j > 0);
+                if (!(ok = wait_issue_PV(1, s, j))) break;
                 tc_commit(&bar_ofull[1]);
                 tc_commit(&bar_vempty[s]);
                 if (jn < n1) {
@@ -327,34 +347,9 @@ __global__ void __launch_bounds__(384, 1)
                 l *= alpha;
                 m = m_new;
             }
-            const float mb = (m == -INFINITY) ? 0.f : m;
-            // p = exp2(S * c - m): the argument as packed two-wide FMAs, the exponential on the
-            // MUFU unit, the row sum in 4 packed accumulators (8 independent chains).  P goes to
-            // tensor memory in two 64-key halves, over S columns already read.
-            const float2 c2 = make_float2(c, c);
-            const float2 nm2 = make_float2(-mb, -mb);
-            float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                             make_float2(0.f, 0.f)};
-#pragma unroll
-            for (int h = 0; h < C::BN / 64; ++h) {
-                uint32_t pk[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int e0 = h * 64 + 2 * i;
-                    const float2 x = ffma2(make_float2(__uint_as_float(s[e0]),
-                                                       __uint_as_float(s[e0 + 1])), c2, nm2);
-                    const float2 e = (i % 4 < FA_FWD_EXP2_FMA_OF_4)
-                                         ? exp2_fma2(x)
-                                         : make_float2(ex2(x.x), ex2(x.y));
-                    acc[i % 4] = fadd2(acc[i % 4], e);
-                    pk[i] = pack_bf16x2(e.x, e.y);
-                }
-                tmem_st32(tS + h * 32, pk);
-            }
-            l += ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
-                 ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
             if (__any_sync(0xffffffffu, grow && j > 0)) {
-                // Rescale this warp's rows of O once the previous P V has landed.
+                // Rescale this warp's rows of O before any of P(j) is released (S(j) done
+                // implies the previous P V of this tile is done: the MMAs run in issue order).
                 ok = mbar_wait(&bar_ofull[t], (j - 1) & 1, p.timeout_ns, abort_flag);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 tc_fence_after();
@@ -375,9 +370,39 @@ __global__ void __launch_bounds__(384, 1)
                     tmem_st32(tO + q * 32, o);
                 }
             }
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&bar_pfull[t]);
+            const float mb = (m == -INFINITY) ? 0.f : m;
+            // p = exp2(S * c - m): the argument as packed two-wide FMAs, the exponential on the
+            // MUFU unit, the row sum in 4 packed accumulators (8 independent chains).  P goes to
+            // tensor memory in P_PARTS parts, over S columns already read; each part is
+            // released to the MMA thread as soon as it is stored.
+            const float2 c2 = make_float2(c, c);
+            const float2 nm2 = make_float2(-mb, -mb);
+            float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                             make_float2(0.f, 0.f)};
+            constexpr int WP = C::BN / 2 / C::P_PARTS;  // packed P words per part
+#pragma unroll
+            for (int part = 0; part < C::P_PARTS; ++part) {
+                uint32_t pk[WP];
+#pragma unroll
+                for (int i = 0; i < WP; ++i) {
+                    const int e0 = part * 2 * WP + 2 * i;
+                    const float2 x = ffma2(make_float2(__uint_as_float(s[e0]),
+                                                       __uint_as_float(s[e0 + 1])), c2, nm2);
+                    const float2 e = (i % 4 < FA_FWD_EXP2_FMA_OF_4)
+                                         ? exp2_fma2(x)
+                                         : make_float2(ex2(x.x), ex2(x.y));
+                    acc[i % 4] = fadd2(acc[i % 4], e);
+                    pk[i] = pack_bf16x2(e.x, e.y);
+                }
+                if constexpr (WP == 32) tmem_st32(tS + part * WP, pk);
+                else tmem_st16(tS + part * WP, pk);
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(part + 1 < C::P_PARTS ? &bar_ppart[t * (C::P_PARTS - 1) + part]
+                                                  : &bar_pfull[t]);
+            }
+            l += ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+                 ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
         }
 
         // ------------------------------------------------------------ epilogue
