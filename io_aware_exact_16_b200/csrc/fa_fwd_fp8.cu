@@ -39,7 +39,7 @@ struct Fp8Cfg {
     static constexpr int SMEM_K = SMEM_Q + TILES * TILE_BYTES;
     static constexpr int SMEM_V = SMEM_K + STAGES * TILE_BYTES;
     static constexpr int SMEM_BAR = SMEM_V + STAGES * TILE_BYTES;
-    static constexpr int NUM_BARS = 1 + 4 * STAGES + 2 + 2 + 2 + 1;
+    static constexpr int NUM_BARS = 1 + 4 * STAGES + 2 + 2 + 2 + 2 + 1;
     static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;
     static constexpr int THREADS = 384;
@@ -143,7 +143,8 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t* bar_sfull = bar_vempty + C::STAGES;  // [2]
     uint64_t* bar_pfull = bar_sfull + 2;            // [2]
     uint64_t* bar_ofull = bar_pfull + 2;            // [2]
-    uint64_t* bar_done = bar_ofull + 2;
+    uint64_t* bar_phalf = bar_ofull + 2;            // [2] P of the block's first 64 keys
+    uint64_t* bar_done = bar_phalf + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SMEM_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::SMEM_MISC + 4);
 
@@ -158,6 +159,7 @@ __global__ void __launch_bounds__(384, 1)
         for (int t = 0; t < 2; ++t) {
             mbar_init(&bar_sfull[t], 1);
             mbar_init(&bar_pfull[t], C::BM);
+            mbar_init(&bar_phalf[t], C::BM);
             mbar_init(&bar_ofull[t], 1);
         }
         mbar_init(bar_done, 1);
@@ -230,15 +232,27 @@ __global__ void __launch_bounds__(384, 1)
                     mma_ss_f8(tmem + C::tm_s(t), sdesc_sw128(qa + kk * 32, 16, 1024),
                               sdesc_sw128(ka + kk * 32, 16, 1024), idS, kk > 0 ? 1u : 0u);
             };
-            // O_t += P_t V: P (e4m3, 4 per column, 8 columns per 32-key step) from tensor
-            // memory, V MN-major (32 key rows = 4096 bytes per step).
-            auto issue_PV = [&](int t, int s, bool accumulate) {
+            // O_t += P_t V over the keys of one half of the block: P (e4m3, 4 per column, 8
+            // columns per 32-key step) from tensor memory, V MN-major (32 key rows = 4096 bytes
+            // per step).  The softmax releases P in two halves, so the first half's MMAs run
+            // while it computes the second half's exponentials.
+            auto issue_PV = [&](int t, int s, bool accumulate, int half) {
                 const uint32_t va = sV + s * C::TILE_BYTES;
 #pragma unroll
-                for (int kk = 0; kk < C::BN / 32; ++kk)
+                for (int kk = half * C::BN / 64; kk < (half + 1) * C::BN / 64; ++kk)
                     mma_ts_f8(tmem + C::tm_o(t), tmem + C::tm_s(t) + kk * 8,
                               sdesc_sw128(va + kk * 4096, C::TILE_BYTES, 1024), idPV,
                               (accumulate || kk > 0) ? 1u : 0u);
+            };
+
+            auto wait_issue_PV = [&](int t, int s, int j) {
+                if (!mbar_wait(&bar_phalf[t], j & 1, p.timeout_ns, abort_flag)) return false;
+                tc_fence_after();
+                issue_PV(t, s, j > 0, 0);
+                if (!mbar_wait(&bar_pfull[t], j & 1, p.timeout_ns, abort_flag)) return false;
+                tc_fence_after();
+                issue_PV(t, s, true, 1);
+                return true;
             };
 
             bool ok = mbar_wait(bar_q, 0, p.timeout_ns, abort_flag);
@@ -259,9 +273,7 @@ __global__ void __launch_bounds__(384, 1)
                 const uint32_t phn = (jn / C::STAGES) & 1;
                 if (!(ok = mbar_wait(&bar_vfull[s], ph, p.timeout_ns, abort_flag))) break;
                 if (j < n0) {
-                    if (!(ok = mbar_wait(&bar_pfull[0], j & 1, p.timeout_ns, abort_flag))) break;
-                    tc_fence_after();
-                    issue_PV(0, s, j > 0);
+                    if (!(ok = wait_issue_PV(0, s, j))) break;
                     tc_commit(&bar_ofull[0]);
                 }
                 if (jn < n1) {
@@ -272,9 +284,7 @@ __global__ void __launch_bounds__(384, 1)
                         tc_commit(&bar_sfull[0]);
                     }
                 }
-                if (!(ok = mbar_wait(&bar_pfull[1], j & 1, p.timeout_ns, abort_flag))) break;
-                tc_fence_after();
-                issue_PV(1, s, j > 0);
+                if (!(ok = wait_issue_PV(1, s, j))) break;
                 tc_commit(&bar_ofull[1]);
                 tc_commit(&bar_vempty[s]);
                 if (jn < n1) {
@@ -341,29 +351,9 @@ __global__ void __launch_bounds__(384, 1)
                 l *= alpha;
                 m = m_new;
             }
-            const float mb = (m == -INFINITY) ? 0.f : m - C::P_OFFSET;
-            const float2 c2 = make_float2(c, c);
-            const float2 nm2 = make_float2(-mb, -mb);
-            float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                             make_float2(0.f, 0.f)};
-            uint32_t pk[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int e0 = 4 * i;
-                const float2 xa = ffma2(make_float2(__uint_as_float(s[e0]),
-                                                    __uint_as_float(s[e0 + 1])), c2, nm2);
-                const float2 xb = ffma2(make_float2(__uint_as_float(s[e0 + 2]),
-                                                    __uint_as_float(s[e0 + 3])), c2, nm2);
-                const float2 ea = make_float2(ex2(xa.x), ex2(xa.y));
-                const float2 eb = make_float2(ex2(xb.x), ex2(xb.y));
-                acc[(2 * i) % 4] = fadd2(acc[(2 * i) % 4], ea);
-                acc[(2 * i + 1) % 4] = fadd2(acc[(2 * i + 1) % 4], eb);
-                pk[i] = pack_e4m3x4(ea.x, ea.y, eb.x, eb.y);
-            }
-            tmem_st32(tS, pk);  // P' (e4m3) over the first 32 columns of S, already read
-            l += ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
-                 ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
             if (__any_sync(0xffffffffu, grow && j > 0)) {
+                // Rescale this warp's rows of O before any of P(j) is released (S(j) done
+                // implies the previous P V of this tile is done: the MMAs run in issue order).
                 ok = mbar_wait(&bar_ofull[t], (j - 1) & 1, p.timeout_ns, abort_flag);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 tc_fence_after();
@@ -384,9 +374,36 @@ __global__ void __launch_bounds__(384, 1)
                     tmem_st32(tO + q * 32, o);
                 }
             }
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&bar_pfull[t]);
+            const float mb = (m == -INFINITY) ? 0.f : m - C::P_OFFSET;
+            const float2 c2 = make_float2(c, c);
+            const float2 nm2 = make_float2(-mb, -mb);
+            float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                             make_float2(0.f, 0.f)};
+            // P' (e4m3) over the first 32 columns of S, already read, in two halves of 64 keys,
+            // each released to the MMA thread as soon as it is stored.
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int e0 = 64 * hh + 4 * i;
+                    const float2 xa = ffma2(make_float2(__uint_as_float(s[e0]),
+                                                        __uint_as_float(s[e0 + 1])), c2, nm2);
+                    const float2 xb = ffma2(make_float2(__uint_as_float(s[e0 + 2]),
+                                                        __uint_as_float(s[e0 + 3])), c2, nm2);
+                    const float2 ea = make_float2(ex2(xa.x), ex2(xa.y));
+                    const float2 eb = make_float2(ex2(xb.x), ex2(xb.y));
+                    acc[(2 * i) % 4] = fadd2(acc[(2 * i) % 4], ea);
+                    acc[(2 * i + 1) % 4] = fadd2(acc[(2 * i + 1) % 4], eb);
+                    pk[i] = pack_e4m3x4(ea.x, ea.y, eb.x, eb.y);
+                }
+                tmem_st16(tS + 16 * hh, pk);
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(hh == 0 ? &bar_phalf[t] : &bar_pfull[t]);
+            }
+            l += ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+                 ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
         }
 
         // ------------------------------------------------------------ epilogue
