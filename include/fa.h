@@ -201,7 +201,7 @@ FA_API fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, cons
  *                  j <= L_b - Nq + i (aligned to the end of the cache); a query that sees no
  *                  key gets O = 0 and lse = -inf.
  *   splits         key ranges per (sequence, cache head) computed by separate CTAs and merged
- *                  by their log-sum-exp; 0 = fa_decode_num_splits(...).  Ranges hold whole key
+ *                  by their log-sum-exp; 0 = fa_decode_num_splits(..., cache_lens != NULL).  Ranges hold whole key
  *                  blocks (64 keys for d <= 128, 128 for d = 256), so the count used may be
  *                  lower than the one requested.
  *   workspace      device, 16-byte aligned, >= fa_decode_workspace_size(B, H, Nq, d, splits)
@@ -209,7 +209,9 @@ FA_API fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, cons
  * d in {64, 128, 256}.  The result is exact for every `splits` (up to rounding: different
  * splits round differently; the same splits give identical bits).
  */
-FA_API int fa_decode_num_splits(int B, int H, int H_kv, int Nq, int N, int d);
+/* Automatic split count; ragged != 0 when per-sequence cache lengths will be passed (more
+ * ranges, so that the longest sequences do not dominate). */
+FA_API int fa_decode_num_splits(int B, int H, int H_kv, int Nq, int N, int d, int ragged);
 FA_API size_t fa_decode_workspace_size(int B, int H, int Nq, int d, int splits);
 FA_API fa_status fa_fwd_decode(const void* q, const void* k_cache, const void* v_cache, void* o,
                                float* lse, const int* cache_lens, int B, int H, int H_kv,

@@ -45,7 +45,7 @@ _lib.fa_fwd_varlen.restype = _i
 _lib.fa_bwd_varlen.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
                                _i, _i, ctypes.c_float, _i, _vp, ctypes.c_size_t, _vp]
 _lib.fa_bwd_varlen.restype = _i
-_lib.fa_decode_num_splits.argtypes = [_i, _i, _i, _i, _i, _i]
+_lib.fa_decode_num_splits.argtypes = [_i, _i, _i, _i, _i, _i, _i]
 _lib.fa_decode_num_splits.restype = _i
 _lib.fa_decode_workspace_size.argtypes = [_i, _i, _i, _i, _i]
 _lib.fa_decode_workspace_size.restype = ctypes.c_size_t
@@ -310,8 +310,10 @@ def forward_fp8(q, k, v, q_descale=None, k_descale=None, v_descale=None, causal:
     return out, lse
 
 
-def decode_num_splits(B: int, H: int, H_kv: int, Nq: int, N: int, d: int) -> int:
-    return int(_lib.fa_decode_num_splits(B, H, H_kv, Nq, N, d))
+def decode_num_splits(B: int, H: int, H_kv: int, Nq: int, N: int, d: int,
+                      ragged: bool = False) -> int:
+    """``fa_decode_num_splits``: ragged = per-sequence cache lengths will be passed."""
+    return int(_lib.fa_decode_num_splits(B, H, H_kv, Nq, N, d, int(bool(ragged))))
 
 
 def decode_workspace_size(B: int, H: int, Nq: int, d: int, splits: int) -> int:
@@ -343,7 +345,7 @@ def decode(q, k_cache, v_cache, cache_lens: Optional[torch.Tensor] = None, causa
     elif lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, Nq) or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous float32 tensor [B, H, Nq]")
     if splits == 0:
-        splits = decode_num_splits(B, H, H_kv, Nq, N, d)
+        splits = decode_num_splits(B, H, H_kv, Nq, N, d, ragged=cache_lens is not None)
     splits = max(1, int(splits))
     need = int(_lib.fa_decode_workspace_size(B, H, Nq, d, splits))  # enough for any count used
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):

@@ -219,7 +219,12 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
 // fewer ranges on ties.  `bk` keys per block, `slots` CTAs resident per wave.  The constant is
 // measured: over split counts of 1 to 64 on five cache shapes it picks the fastest one each
 // time (one block of fixed cost picked up to 9 % slower counts).
-int decode_splits(int B, int H_kv, int n_mt, int N, int bk, int slots) {
+// With per-sequence lengths (`ragged`, known only on the device) the waves model overrates a
+// few long ranges, because the short sequences' CTAs finish early; there the count is at least
+// ceil(4 slots / pairs), which keeps the longest range near half of one slot's share of the
+// work when lengths average N / 2 (on four ragged batches this lands on or next to the fastest
+// count; the waves model alone was up to 1.6x slower).
+int decode_splits(int B, int H_kv, int n_mt, int N, int bk, int slots, bool ragged) {
     const int nblk = (N + bk - 1) / bk;
     const long long base = (long long)B * H_kv * n_mt;
     int best = 1;
@@ -233,6 +238,10 @@ int decode_splits(int B, int H_kv, int n_mt, int N, int bk, int slots) {
             best_cost = cost;
             best = s;
         }
+    }
+    if (ragged) {
+        const long long floor_s = (4LL * slots + base - 1) / base;
+        if (best < floor_s) best = (int)(floor_s < nblk ? floor_s : nblk);
     }
     return best;
 }
@@ -443,7 +452,7 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, const float* q
     return FA_OK;
 }
 
-int fa_decode_num_splits(int B, int H, int H_kv, int Nq, int N, int d) {
+int fa_decode_num_splits(int B, int H, int H_kv, int Nq, int N, int d, int ragged) {
     if (check_decode(B, H, H_kv, Nq, N, d, 1.0f, 0) != FA_OK) return 0;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) {
@@ -452,7 +461,8 @@ int fa_decode_num_splits(int B, int H, int H_kv, int Nq, int N, int d) {
             sms = v;
     }
     const int n_mt = ((H / H_kv) * Nq + 127) / 128;
-    return decode_splits(B, H_kv, n_mt, N, decode_block_keys(d), sms * decode_ctas_per_sm(d));
+    return decode_splits(B, H_kv, n_mt, N, decode_block_keys(d), sms * decode_ctas_per_sm(d),
+                         ragged != 0);
 }
 
 size_t fa_decode_workspace_size(int B, int H, int Nq, int d, int splits) {
@@ -482,7 +492,8 @@ fa_status fa_fwd_decode(const void* q, const void* k_cache, const void* v_cache,
     const int bk = decode_block_keys(d);
     const int nblk = (N + bk - 1) / bk;
     if (splits == 0)
-        splits = decode_splits(B, H_kv, n_mt, N, bk, dev->num_sms * decode_ctas_per_sm(d));
+        splits = decode_splits(B, H_kv, n_mt, N, bk, dev->num_sms * decode_ctas_per_sm(d),
+                               cache_lens != nullptr);
     if (splits > nblk) splits = nblk;
     const int bps = (nblk + splits - 1) / splits;
     splits = (nblk + bps - 1) / bps;  // ranges that actually hold keys

@@ -148,3 +148,12 @@ def test_decode_split_heuristic_and_workspace_size():
     o_bytes = (5 * rows * 128 * 4 + 255) // 256 * 256
     assert fa.decode_workspace_size(2, 4, 3, 128, 5) == o_bytes + 5 * rows * 4
     assert fa.decode_num_splits(1, 4, 3, 1, 100, 128) == 0  # H_kv must divide H
+    # per-sequence lengths: at least ceil(4 x 296 slots / pairs) ranges, within the key blocks
+    for (B, H, H_kv, Nq, N, d) in ((32, 32, 8, 1, 8192, 128), (8, 32, 8, 1, 32768, 128),
+                                   (128, 32, 8, 1, 4096, 128), (16, 32, 8, 1, 16384, 128),
+                                   (1, 8, 8, 1, 64, 64)):
+        u = fa.decode_num_splits(B, H, H_kv, Nq, N, d)
+        r = fa.decode_num_splits(B, H, H_kv, Nq, N, d, ragged=True)
+        nblk = (N + 63) // 64
+        assert r == max(u, min(nblk, -(-4 * 296 // (B * H_kv))))
+    assert fa.decode_num_splits(32, 32, 8, 1, 8192, 128, ragged=True) == 5
