@@ -104,3 +104,47 @@ def test_long_context_sampled_rows(N):
     for h in range(w.H):
         O_ref, lse_ref = oracle.head_fwd_rows(inp.q[0, h], inp.k[0, h], inp.v[0, h], rows, w.scale, True)
         assert_fwd_close(O[0, h, rows], lse[0, h, rows], O_ref, lse_ref, f"head {h} rows")
+
+
+@pytest.mark.parametrize("N", [16384, 32768])
+def test_long_context_longer_sampled_rows(N):
+    """Long-context config at 16K and 32K: 256 seeded rows of every head (plus the first and
+    last rows and tile edges).  Whole heads would need an N x N fp64 score matrix on the host
+    (8.6 GB at 32K), so these sizes check sampled rows only."""
+    w = workloads.long_context(N)
+    inp, O, lse = run_fwd(w)
+    rows = sorted(set(workloads.seeded_sample(w.seed + 2, N, 250) +
+                      [0, 127, 128, 255, 256, N // 2, N - 129, N - 128, N - 1]))
+    for h in range(w.H):
+        O_ref, lse_ref = oracle.head_fwd_rows(inp.q[0, h], inp.k[0, h], inp.v[0, h], rows, w.scale, True)
+        assert_fwd_close(O[0, h, rows], lse[0, h, rows], O_ref, lse_ref, f"N {N} head {h} rows")
+
+
+def test_forward_memory_is_inputs_plus_outputs():
+    """The forward allocates nothing on the device: with O and lse preallocated, the peak
+    allocation over the call equals what was resident before it (Q, K, V, O, lse), which
+    doubles with N (long-context config, 8K -> 16K -> 32K); the N x N score matrix (16 N^2
+    bytes in bf16 for 16 heads) is never materialised."""
+    fa = _fa()
+    dev = torch.device("cuda", 0)
+    totals = []
+    for N in (8192, 16384, 32768):
+        w = workloads.long_context(N)
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        q, k, v = (torch.randn(1, w.H, N, w.d, device=dev).to(torch.bfloat16) for _ in range(3))
+        o = torch.empty_like(q)
+        lse = torch.empty((1, w.H, N), dtype=torch.float32, device=dev)
+        fa.forward(q, k, v, causal=True, out=o, lse=lse)  # first call: per-device state
+        torch.cuda.synchronize()
+        before = torch.cuda.memory_allocated(dev)
+        torch.cuda.reset_peak_memory_stats(dev)
+        fa.forward(q, k, v, causal=True, out=o, lse=lse)
+        torch.cuda.synchronize()
+        assert fa.check_device_error() == 0
+        assert torch.cuda.max_memory_allocated(dev) == before
+        io_bytes = 4 * w.H * N * w.d * 2 + w.H * N * 4
+        totals.append(io_bytes)
+        assert sum(t.numel() * t.element_size() for t in (q, k, v, o, lse)) == io_bytes
+        del q, k, v, o, lse
+    assert totals[1] == 2 * totals[0] and totals[2] == 2 * totals[1]
