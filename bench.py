@@ -107,6 +107,12 @@ def dram_traffic(kernel: str, workload: str) -> float | None:
     return float(entry["dram_bytes_per_launch"])
 
 
+def _pct(sorted_vals, q):
+    """q-th percentile (nearest rank) of an ascending list."""
+    i = min(len(sorted_vals) - 1, max(0, int(round(q / 100 * (len(sorted_vals) - 1)))))
+    return sorted_vals[i]
+
+
 class ClockSampler:
     """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
 
@@ -256,6 +262,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     elapsed_ms = start.elapsed_time(end)
     fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
     bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    step_ms = sorted(e[0].elapsed_time(e[2]) for e in ev)  # per step, for the spread
     fwd_kernel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in kev)
     bwd_kernel_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in kev)
     status = fa.check_device_error(dev)
@@ -361,7 +368,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
         "passes": {"fwd_ms": round(fwd_ms, 4), "bwd_ms": round(bwd_ms, 4),
                    "fwd_tflops": round(fwd_tflops, 2), "bwd_tflops": round(bwd_tflops, 2),
                    "fwd_pct_of_2250": round(100 * fwd_tflops / NOMINAL_PEAK_TFLOPS, 2),
-                   "bwd_pct_of_2250": round(100 * bwd_tflops / NOMINAL_PEAK_TFLOPS, 2)},
+                   "bwd_pct_of_2250": round(100 * bwd_tflops / NOMINAL_PEAK_TFLOPS, 2),
+                   "step_ms_p10_p50_p90": [round(_pct(step_ms, q), 4) for q in (10, 50, 90)]},
         "roofline": {
             "kernel": "fa_bwd_kernel (fused backward: all five backward GEMMs)",
             "bound": "tensor", "achieved": round(bwd_kernel_tflops, 2),
