@@ -99,11 +99,10 @@ DeviceState* current_device(fa_status* st) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// d = 256 has a forward kernel only (`fwd`).
-fa_status check_common(int B, int H, int N, int d, float scale, bool fwd = false) {
+fa_status check_common(int B, int H, int N, int d, float scale) {
     if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
     if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
-    if (d != 64 && d != 128 && !(fwd && d == 256)) return FA_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
     if (B > 65535 || H > 65535) return FA_ERR_INVALID_ARG;
     const long long elems = (long long)B * H * N * d;
     if (elems >= (1ll << 31)) return FA_ERR_INVALID_ARG;
@@ -154,18 +153,21 @@ bool make_fp8_map(CUtensorMap* map, const void* base, int N, int BHx) {
 
 namespace {
 
-// Tensor map of a user tensor with Hx heads: head-major [B, Hx, N, d] or packed [T, Hx, d].
+// Tensor map of a user tensor with Hx heads: head-major [B, Hx, N, d] or packed [T, Hx, d];
+// boxes of 64 columns x `rows` rows.
 bool user_map(CUtensorMap* map, const void* base, int d, int B, int Hx, int N, int T,
-              bool packed) {
-    return packed ? make_bf16_map_packed(map, base, d, Hx, T, 128)
-                  : make_bf16_map(map, base, d, N, B * Hx, 128);
+              bool packed, int rows = 128) {
+    return packed ? make_bf16_map_packed(map, base, d, Hx, T, rows)
+                  : make_bf16_map(map, base, d, N, B * Hx, rows);
 }
 
-// Checks shared by the head-major and packed entry points; T = 0 for head-major.
+// Checks shared by the head-major and packed entry points; T = 0 for head-major.  The d = 256
+// backward runs head-major only (`fwd` false).
 fa_status check_layout(int B, int H, int H_kv, int N, int d, float scale, const int* seqlens,
                        const int* cu_seqlens, int T, bool fwd) {
-    fa_status st = check_common(B, H, N, d, scale, fwd);
+    fa_status st = check_common(B, H, N, d, scale);
     if (st != FA_OK) return st;
+    if (!fwd && d == 256 && cu_seqlens) return FA_ERR_UNSUPPORTED;
     if (H_kv < 1 || H_kv > H || H % H_kv != 0) return FA_ERR_INVALID_ARG;
     if (seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u)) return FA_ERR_INVALID_ARG;
     if (cu_seqlens) {
@@ -371,8 +373,11 @@ static fa_status bwd_impl(const void* q, const void* k, const void* v, const voi
 
     const bool packed = cu_seqlens != nullptr;
     CUtensorMap tq, tk, tv, tdo;
-    if (!user_map(&tq, q, d, B, H, N, T, packed) || !user_map(&tk, k, d, B, H_kv, N, T, packed) ||
-        !user_map(&tv, v, d, B, H_kv, N, T, packed) || !user_map(&tdo, dO, d, B, H, N, T, packed))
+    const int q_rows = d == 256 ? 64 : 128;  // query rows per backward step
+    if (!user_map(&tq, q, d, B, H, N, T, packed, q_rows) ||
+        !user_map(&tk, k, d, B, H_kv, N, T, packed) ||
+        !user_map(&tv, v, d, B, H_kv, N, T, packed) ||
+        !user_map(&tdo, dO, d, B, H, N, T, packed, q_rows))
         return FA_ERR_CUDA;
     cudaEvent_t ev0, ev1;
     take_timing_events(&ev0, &ev1);

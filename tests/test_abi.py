@@ -79,8 +79,8 @@ def test_backward_rejects_bad_arguments_and_short_workspace_without_a_device():
                           ctypes.c_float(0.125), 0, None, ws, ws_bytes, None)
 
     assert bwd(d=80) == fa.FA_ERR_UNSUPPORTED
-    assert bwd(d=256) == fa.FA_ERR_UNSUPPORTED      # head dim 256 has a forward kernel only
-    assert fa.bwd_workspace_size(1, 1, 8, 256) == 0
+    assert fa.bwd_workspace_size(1, 1, 8, 256) > need
+    assert bwd(d=256) == fa.FA_ERR_WORKSPACE        # d = 256 needs its own, larger workspace
     assert bwd(ptr=None) == fa.FA_ERR_INVALID_ARG
     assert bwd(ws=None) == fa.FA_ERR_WORKSPACE
     assert bwd(ws_bytes=need - 1) == fa.FA_ERR_WORKSPACE

@@ -1,12 +1,13 @@
-"""GPU parity of the head-dimension-256 forward kernel (``fa_fwd`` / ``fa_fwd_gqa`` /
-``fa_fwd_varlen`` with d = 256) against the fp64 oracle on the same seeded bf16 inputs."""
+"""GPU parity of the head-dimension-256 kernels (``fa_fwd`` / ``fa_fwd_gqa`` / ``fa_fwd_varlen``
+and ``fa_bwd`` / ``fa_bwd_gqa`` with d = 256) against the fp64 oracle on the same seeded bf16
+inputs."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
 import workloads
-from tests.gpu_helpers import assert_fwd_close, to_np
+from tests.gpu_helpers import assert_fwd_close, assert_grad_close, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -81,15 +82,70 @@ def test_d256_packed_sequences():
     assert_fwd_close(to_np(O), to_np(lse), O_ref, lse_ref, "packed d256")
 
 
-def test_d256_forward_is_deterministic_and_backward_unsupported():
-    fa = _fa()
+def test_d256_forward_is_deterministic():
     w = workloads.custom(2, 2, 700, 256, False, seed=8300)
     inp, O1, l1 = run_fwd(w)
     _, O2, l2 = run_fwd(w, inp)
     np.testing.assert_array_equal(O1, O2)
     np.testing.assert_array_equal(l1, l2)
+
+
+def run_fwd_bwd(w: workloads.Workload, inp=None):
+    fa = _fa()
+    inp = inp or workloads.make_inputs(w)
     dev = torch.device("cuda", 0)
-    q = inp.q.to(dev)
+    q, k, v, do = (t.to(dev) for t in (inp.q, inp.k, inp.v, inp.do))
+    sl = inp.seqlens.to(dev) if inp.seqlens is not None else None
+    O, lse = fa.forward(q, k, v, causal=w.causal, seqlens=sl, scale=w.scale)
+    dq, dk, dv = fa.backward(q, k, v, O, do, lse, causal=w.causal, seqlens=sl, scale=w.scale)
+    assert fa.check_device_error() == 0
+    assert dk.shape == k.shape and dv.shape == v.shape
+    return inp, {"o": to_np(O), "lse": to_np(lse), "dq": to_np(dq), "dk": to_np(dk),
+                 "dv": to_np(dv)}
+
+
+BWD = [
+    # (B, H, H_kv, N, causal, pad_range): one step, ragged tails across 64-query steps and
+    # 128-key blocks, N = 1, padding, grouped-query and multi-query heads
+    (1, 1, 1, 1, False, None),
+    (1, 2, 2, 128, True, None),
+    (1, 2, 2, 100, False, None),
+    (2, 2, 2, 300, True, None),
+    (2, 3, 3, 257, False, None),
+    (3, 2, 2, 384, False, (1, 384)),
+    (2, 2, 2, 520, True, (100, 520)),
+    (2, 4, 2, 384, True, None),
+    (1, 6, 1, 300, False, None),
+    (1, 2, 2, 1000, True, None),
+]
+
+
+@pytest.mark.parametrize("shape", BWD, ids=lambda s: "B{}H{}kv{}N{}{}{}".format(
+    s[0], s[1], s[2], s[3], "c" if s[4] else "", "pad" if s[5] else ""))
+def test_d256_backward_matches_oracle(shape):
+    B, H, H_kv, N, causal, pad = shape
+    w = workloads.custom(B, H, N, 256, causal, seed=8400 + N + H, pad_range=pad, H_kv=H_kv)
+    inp, got = run_fwd_bwd(w)
+    ref = oracle.attention_bwd_gqa(inp.q, inp.k, inp.v, inp.do, w.scale, causal, inp.seqlens)
+    assert_fwd_close(got["o"], got["lse"], ref["o"], ref["lse"], str(shape))
+    for name in ("dq", "dk", "dv"):
+        assert_grad_close(got[name], ref[name], name, str(shape))
+
+
+def test_d256_backward_is_bitwise_deterministic():
+    w = workloads.custom(2, 4, 700, 256, True, seed=8500, H_kv=2)
+    inp = workloads.make_inputs(w)
+    _, a = run_fwd_bwd(w, inp)
+    _, b = run_fwd_bwd(w, inp)
+    for name in ("dq", "dk", "dv"):
+        np.testing.assert_array_equal(a[name], b[name], err_msg=name)
+
+
+def test_d256_packed_backward_unsupported():
+    fa = _fa()
+    dev = torch.device("cuda", 0)
+    x = torch.zeros((10, 2, 256), dtype=torch.bfloat16, device=dev)
+    cu = torch.tensor([0, 4, 10], dtype=torch.int32, device=dev)
     with pytest.raises(fa.FAError) as e:
-        fa.backward(q, q, q, q, q, torch.zeros((2, 2, 700), device=dev))
+        fa.backward_varlen(x, x, x, x, x, torch.zeros((2, 10), device=dev), cu, 6)
     assert e.value.status == fa.FA_ERR_UNSUPPORTED
