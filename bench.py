@@ -8,7 +8,7 @@ B = 16384 / N = 4 per GPU (the size at which the throughput targets are stated).
 FLOP accounting: forward 4*B*H*N^2*d (halved when causal), backward 2.5x the forward.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
-    python bench.py --row fwd-d256|fwd-fp8|decode|varlen [...]   (the further entry points)
+    python bench.py --row fwd-d256|bwd-d256|fwd-fp8|decode|varlen [...]   (the further entry points)
 
 With N > 1 launch one process per GPU with torch.distributed.run; each rank runs its own
 batch of the same shape (weak scaling, no collective on the data path) and rank 0 prints one
@@ -76,9 +76,10 @@ def load_peaks() -> tuple[dict, str]:
 
 KERNEL_SOURCES = {
     "fa_fwd_kernel": ("fa_fwd.cu", "sm100.cuh", "fa_internal.h"),
-    "fa_bwd_kernel": ("fa_bwd.cu", "sm100.cuh", "fa_internal.h"),
+    "fa_bwd_kernel": ("fa_bwd.cu", "fa_bwd_common.cuh", "sm100.cuh", "fa_internal.h"),
     "fa_fwd_d256_kernel": ("fa_fwd_d256.cu", "sm100.cuh", "fa_internal.h"),
     "fa_fwd_fp8_kernel": ("fa_fwd_fp8.cu", "fa_fwd_fp8.h", "sm100.cuh", "fa_internal.h"),
+    "fa_bwd_d256_kernel": ("fa_bwd_d256.cu", "fa_bwd_common.cuh", "sm100.cuh", "fa_internal.h"),
     "fa_decode_kernel": ("fa_decode.cu", "fa_decode.h", "sm100.cuh", "fa_internal.h"),
 }
 
@@ -533,6 +534,42 @@ def row_fwd_d256(rank: int, dev) -> Row:
                d2h=[_pinned_pair(o)], launches=1, cpu=cpu, traffic_key="fa_fwd_d256_kernel")
 
 
+def row_bwd_d256(rank: int, dev) -> Row:
+    import io_aware_exact_16_b200 as fa
+    import oracle
+    w = workloads.Workload("d256 bwd non-causal B2 H16 N4096 d256", 2, 16, 4096, 256, False,
+                           1080 + 7919 * rank)
+    inp = workloads.make_inputs(w)
+    q, k, v, do = (t.to(dev) for t in (inp.q, inp.k, inp.v, inp.do))
+    o, lse = fa.forward(q, k, v, scale=w.scale)
+    dq, dk, dv = (torch.empty_like(t) for t in (q, k, v))
+    ws = torch.empty(fa.bwd_workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+    flops = 2.5 * 4.0 * w.B * w.H * w.N * w.N * w.d  # five GEMMs; the recompute is not counted
+    bf16, _, src = _peaks()
+
+    def cpu():
+        heads = workloads.seeded_sample(w.seed + 5, w.B * w.H, 1)
+        t0 = time.perf_counter()
+        for flat in heads:
+            b, h = divmod(flat, w.H)
+            oracle.head_bwd(inp.q[b, h], inp.k[b, h], inp.v[b, h], inp.do[b, h], w.scale, False)
+        return {"amount": flops / (w.B * w.H) * len(heads), "seconds": time.perf_counter() - t0,
+                "sample": f"fp64 C oracle backward on {len(heads)} of {w.B * w.H} heads"}
+
+    o_h, lse_h = o.cpu().pin_memory(), lse.cpu().pin_memory()
+    return Row(config={"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                       "causal": False, "l2": "Q,K,V,O,dO,dQ,dK,dV are 67 MB each"},
+               metric="bf16 attention backward TFLOP/s at head dim 256", unit="TFLOP/s",
+               dtype="bf16", amount=flops, kernel="fa_bwd_d256_kernel", kernel_amount=flops,
+               bound="tensor", peak=bf16, peak_source=f"{src} bf16 sustained",
+               step=lambda mark: (mark(), fa.backward(q, k, v, o, do, lse, scale=w.scale, dq=dq,
+                                                      dk=dk, dv=dv, workspace=ws)),
+               h2d=[(q, inp.q.pin_memory()), (k, inp.k.pin_memory()), (v, inp.v.pin_memory()),
+                    (do, inp.do.pin_memory()), (o, o_h), (lse, lse_h)],
+               d2h=[_pinned_pair(dq), _pinned_pair(dk), _pinned_pair(dv)], launches=3, cpu=cpu,
+               traffic_key="fa_bwd_d256_kernel")
+
+
 def row_fwd_fp8(rank: int, dev) -> Row:
     import io_aware_exact_16_b200 as fa
     import oracle
@@ -652,7 +689,7 @@ def row_varlen(rank: int, dev) -> Row:
                d2h=[_pinned_pair(t) for t in (o, dq, dk, dv)], launches=4, cpu=cpu)
 
 
-ROWS = {"fwd-d256": row_fwd_d256, "fwd-fp8": row_fwd_fp8, "decode": row_decode,
+ROWS = {"fwd-d256": row_fwd_d256, "bwd-d256": row_bwd_d256, "fwd-fp8": row_fwd_fp8, "decode": row_decode,
         "varlen": row_varlen}
 
 

@@ -16,10 +16,10 @@
  * ---------------------------------------
  * Layout.     Q, K, V, O, dO, dQ, dK, dV are bf16, contiguous, shape [B, H, N, d]
  *             (row-major: d fastest, then N, then H, then B).  lse is fp32 [B, H, N].
- * Sizes.      B >= 1, H >= 1, 1 <= N, d in {64, 128}, and for the forward entry points also
- *             d = 256 (FlashAttention (DE), "FlashAttention-2 (2023)": heads of size 256; the
- *             backward entry points return FA_ERR_UNSUPPORTED for it); B*H*N*d must fit in
- *             2^31 elements.
+ * Sizes.      B >= 1, H >= 1, 1 <= N, d in {64, 128, 256} (FlashAttention (DE),
+ *             "FlashAttention-2 (2023)": heads of size 256); fa_bwd_varlen returns
+ *             FA_ERR_UNSUPPORTED for d = 256 (its backward runs head-major only) and
+ *             fa_bwd_noalloc for anything but 64 and 128; B*H*N*d must fit in 2^31 elements.
  * Mask.       causal != 0 hides key j from query i when j > i (top-left alignment, N queries
  *             and N keys).  seqlens, when not NULL, is a DEVICE int32 array of B key lengths
  *             L_b with 1 <= L_b <= N: keys j >= L_b of batch b are hidden from every query.
@@ -61,7 +61,7 @@ typedef struct CUstream_st* fa_stream_t;
 typedef enum {
     FA_OK = 0,
     FA_ERR_INVALID_ARG = 1,  /* a NULL/misaligned pointer, a size or scale out of range      */
-    FA_ERR_UNSUPPORTED = 2,  /* head dim not 64/128 (256: forward only), or not an sm_100 GPU */
+    FA_ERR_UNSUPPORTED = 2,  /* head dim not 64/128/256 for this entry point, or not an sm_100 GPU */
     FA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed (launch, tensor map, ...)  */
     FA_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up (reported by the flag)   */
     FA_ERR_WORKSPACE = 5     /* fa_bwd: workspace NULL, misaligned or smaller than required */
