@@ -17,9 +17,8 @@
  * Layout.     Q, K, V, O, dO, dQ, dK, dV are bf16, contiguous, shape [B, H, N, d]
  *             (row-major: d fastest, then N, then H, then B).  lse is fp32 [B, H, N].
  * Sizes.      B >= 1, H >= 1, 1 <= N, d in {64, 128, 256} (FlashAttention (DE),
- *             "FlashAttention-2 (2023)": heads of size 256); fa_bwd_varlen returns
- *             FA_ERR_UNSUPPORTED for d = 256 (its backward runs head-major only) and
- *             fa_bwd_noalloc for anything but 64 and 128; B*H*N*d must fit in 2^31 elements.
+ *             "FlashAttention-2 (2023)": heads of size 256; fa_bwd_noalloc takes 64 and 128
+ *             only); B*H*N*d must fit in 2^31 elements.
  * Mask.       causal != 0 hides key j from query i when j > i (top-left alignment, N queries
  *             and N keys).  seqlens, when not NULL, is a DEVICE int32 array of B key lengths
  *             L_b with 1 <= L_b <= N: keys j >= L_b of batch b are hidden from every query.

@@ -161,13 +161,12 @@ bool user_map(CUtensorMap* map, const void* base, int d, int B, int Hx, int N, i
                   : make_bf16_map(map, base, d, N, B * Hx, rows);
 }
 
-// Checks shared by the head-major and packed entry points; T = 0 for head-major.  The d = 256
-// backward runs head-major only (`fwd` false).
+// Checks shared by the head-major and packed entry points; T = 0 for head-major.
 fa_status check_layout(int B, int H, int H_kv, int N, int d, float scale, const int* seqlens,
                        const int* cu_seqlens, int T, bool fwd) {
+    (void)fwd;  // every head dim has both passes in both layouts
     fa_status st = check_common(B, H, N, d, scale);
     if (st != FA_OK) return st;
-    if (!fwd && d == 256 && cu_seqlens) return FA_ERR_UNSUPPORTED;
     if (H_kv < 1 || H_kv > H || H % H_kv != 0) return FA_ERR_INVALID_ARG;
     if (seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u)) return FA_ERR_INVALID_ARG;
     if (cu_seqlens) {

@@ -631,7 +631,7 @@ cudaError_t launch_bwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 
 }  // namespace
 
-// d = 256 (fa_bwd_d256.cu; head-major only): Q and dO maps with 64-row boxes.
+// d = 256 (fa_bwd_d256.cu, both layouts): Q and dO maps with 64-row boxes.
 cudaError_t launch_bwd_d256(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream,
                             cudaEvent_t ev_start, cudaEvent_t ev_stop);

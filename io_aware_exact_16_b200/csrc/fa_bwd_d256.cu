@@ -1,4 +1,5 @@
-// fa_bwd_d256.cu -- exact-attention backward pass for head dim 256 (sm_100a).
+// fa_bwd_d256.cu -- exact-attention backward pass for head dim 256 (sm_100a), head-major and
+// packed layouts.
 //
 // The same computation as fa_bwd.cu (recompute P from the forward's log-sum-exp, then
 // dV = P^T dO, dS = P * (dP - D), dK = scale dS^T Q, dQ = scale dS K; flash-attention glossary
@@ -69,6 +70,7 @@ struct Bwd256 {
                   "swizzled tiles must start on 1024-byte boundaries");
 };
 
+template <bool PACKED>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_d256_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
@@ -107,13 +109,23 @@ __global__ void __launch_bounds__(512, 1)
     const int b = bhk / p.H_kv;
     const int G = p.H / p.H_kv;             // query heads sharing this key/value head
     const int bh_first = b * p.H + (bhk % p.H_kv) * G;
+    constexpr bool packed = PACKED;
     const SeqExtent ext = sequence_extent(p, b, threadIdx.x == 0 && j == 0 && hd == 0 &&
-                                                    bhk % p.H_kv == 0, false);
+                                                    bhk % p.H_kv == 0, packed);
     const int L = ext.L;
     const int n_q = (ext.Lq + C::BM - 1) / C::BM;  // 64-row query blocks
     const int k0 = j * C::BN;
 
+    // TMA coordinates (y, z) of row n of query head qh (= b*H + h) and of this key/value head:
+    // head-major (n, head), packed (head within the sequence, t0 + n).
+    auto q_y = [&](int qh, int n) { return packed ? qh - b * p.H : n; };
+    auto q_z = [&](int qh, int n) { return packed ? ext.t0 + n : qh; };
+    const int kv_y = packed ? bhk % p.H_kv : k0;
+    const int kv_z = packed ? ext.t0 + k0 : bhk;
+
     if (k0 >= L) {
+        // Packed: these rows belong to no key of this sequence; nothing to write.
+        if (packed) return;
         // Every key of this block is padding: dK = dV = 0 (this CTA's feature half).
         const int rows = min(C::BN, p.N - k0);
         __nv_bfloat16* dk = reinterpret_cast<__nv_bfloat16*>(p.dk) + ((size_t)bhk * p.N + k0) * D;
@@ -218,8 +230,8 @@ __global__ void __launch_bounds__(512, 1)
         prefetch_tensormap(&tmDO);
         mbar_arrive_expect_tx(bar_kv, 2 * C::KCH * C::KV_CHUNK);
         for (int c = 0; c < C::KCH; ++c) {
-            tma_load_3d(smem + C::SMEM_K + c * C::KV_CHUNK, &tmK, bar_kv, c * 64, k0, bhk);
-            tma_load_3d(smem + C::SMEM_V + c * C::KV_CHUNK, &tmV, bar_kv, c * 64, k0, bhk);
+            tma_load_3d(smem + C::SMEM_K + c * C::KV_CHUNK, &tmK, bar_kv, c * 64, kv_y, kv_z);
+            tma_load_3d(smem + C::SMEM_V + c * C::KV_CHUNK, &tmV, bar_kv, c * 64, kv_y, kv_z);
         }
         int it = 0;
         Step st{0, 0};
@@ -230,8 +242,10 @@ __global__ void __launch_bounds__(512, 1)
             if (!mbar_wait(bar_qempty, (it & 1) ^ 1, p.timeout_ns, abort_flag)) { fail(); break; }
             mbar_arrive_expect_tx(bar_qfull, 2 * C::KCH * C::Q_CHUNK);
             for (int c = 0; c < C::KCH; ++c) {
-                tma_load_3d(smem + C::SMEM_Q + c * C::Q_CHUNK, &tmQ, bar_qfull, c * 64, q0, qh);
-                tma_load_3d(smem + C::SMEM_DO + c * C::Q_CHUNK, &tmDO, bar_qfull, c * 64, q0, qh);
+                tma_load_3d(smem + C::SMEM_Q + c * C::Q_CHUNK, &tmQ, bar_qfull, c * 64,
+                            q_y(qh, q0), q_z(qh, q0));
+                tma_load_3d(smem + C::SMEM_DO + c * C::Q_CHUNK, &tmDO, bar_qfull, c * 64,
+                            q_y(qh, q0), q_z(qh, q0));
             }
         }
         // Do not leave while our copies may still be landing in shared memory.
@@ -321,11 +335,16 @@ __global__ void __launch_bounds__(512, 1)
         // lse values, 64..127 the D values); -inf / 0 past N so those queries get P = 0.  The
         // global load is issued one step ahead and stored at the end of the step.
         float staged = 0.f;
+        // lse of query head bh_first + g, position q: lse[lse_base + g * lse_hstride + q].
+        const size_t lse_hstride = packed ? (size_t)p.T : (size_t)p.N;
+        const size_t lse_base = lse_of(packed, b, bh_first - b * p.H, p.H, p.N, p.T, ext.t0, 0);
         auto load_vectors = [&](Step s) {
             const int q = q_block(s) * C::BM + (ct & 63);
-            const size_t row = (size_t)q_head(s) * p.N + q;
-            if (ct < 64) staged = q < ext.Lq ? -p.lse[row] * kLog2e : -INFINITY;
-            else if (ct < 128) staged = q < ext.Lq ? p.Dvec[row] : 0.f;
+            if (ct < 64)
+                staged = q < ext.Lq ? -p.lse[lse_base + (size_t)s.g * lse_hstride + q] * kLog2e
+                                    : -INFINITY;
+            else if (ct < 128)
+                staged = q < ext.Lq ? p.Dvec[(size_t)q_head(s) * p.N + q] : 0.f;
         };
         auto store_vectors = [&](int it) {
             if (ct < 64) s_lse2[(it & 1) * C::BM + ct] = staged;
@@ -434,8 +453,10 @@ __global__ void __launch_bounds__(512, 1)
         if (ok) ok = mbar_wait(bar_done, 0, p.timeout_ns, abort_flag);  // every MMA finished
         if (__all_sync(0xffffffffu, ok)) {
             tc_fence_after();
-            const bool in_range = kidx < p.N;
-            const size_t off = ((size_t)bhk * p.N + (in_range ? kidx : 0)) * D + hd * C::DH;
+            const bool in_range = kidx < (packed ? L : p.N);
+            const size_t off =
+                row_of(packed, b, bhk % p.H_kv, p.H_kv, p.N, ext.t0, in_range ? kidx : 0) * D +
+                hd * C::DH;
             const uint32_t col0 = h ? C::TM_DK : C::TM_DV;
             const float mul = h ? p.scale : 1.0f;
             __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(h ? p.dk : p.dv) + off;
@@ -479,17 +500,22 @@ cudaError_t launch_bwd_d256(const CUtensorMap& tq, const CUtensorMap& tk, const 
     using C = Bwd256;
     static bool configured = false;  // attribute set once per process (idempotent if raced)
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(fa_bwd_d256_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::SMEM_BYTES);
-        if (e != cudaSuccess) return e;
+        for (auto kern : {fa_bwd_d256_kernel<false>, fa_bwd_d256_kernel<true>}) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 C::SMEM_BYTES);
+            if (e != cudaSuccess) return e;
+        }
         configured = true;
     }
     const dim3 chunks(p.N_pad / 128, p.B * p.H);
     const int n_kv = (p.N + C::BN - 1) / C::BN;
     fa_bwd_pre_kernel<256><<<chunks, 256, 0, stream>>>(p);
     if (ev_start) cudaEventRecord(ev_start, stream);
-    fa_bwd_d256_kernel<<<p.B * p.H_kv * n_kv * 2, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
+    const unsigned grid = (unsigned)(p.B * p.H_kv * n_kv * 2);
+    if (p.cu_seqlens != nullptr)
+        fa_bwd_d256_kernel<true><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
+    else
+        fa_bwd_d256_kernel<false><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
     if (ev_stop) cudaEventRecord(ev_stop, stream);
     fa_bwd_dq_kernel<256><<<chunks, 256, 0, stream>>>(p);
     return cudaGetLastError();

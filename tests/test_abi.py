@@ -113,7 +113,7 @@ def test_gqa_and_varlen_reject_bad_arguments_without_a_device():
         fa.FA_ERR_INVALID_ARG
     assert lib.fa_fwd_varlen(16, 16, 16, 16, 16, 18, 2, 8, 16, 4, 4, 64, f, 0, None) == \
         fa.FA_ERR_INVALID_ARG
-    assert lib.fa_bwd_varlen(16, 16, 16, 16, 16, 16, 16, 16, 16, 16, 2, 8, 16, 4, 4, 256, f, 0,
+    assert lib.fa_bwd_varlen(16, 16, 16, 16, 16, 16, 16, 16, 16, 16, 2, 8, 16, 4, 4, 96, f, 0,
                              16, 1 << 20, None) == fa.FA_ERR_UNSUPPORTED
 
 

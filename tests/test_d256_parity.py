@@ -139,13 +139,3 @@ def test_d256_backward_is_bitwise_deterministic():
     _, b = run_fwd_bwd(w, inp)
     for name in ("dq", "dk", "dv"):
         np.testing.assert_array_equal(a[name], b[name], err_msg=name)
-
-
-def test_d256_packed_backward_unsupported():
-    fa = _fa()
-    dev = torch.device("cuda", 0)
-    x = torch.zeros((10, 2, 256), dtype=torch.bfloat16, device=dev)
-    cu = torch.tensor([0, 4, 10], dtype=torch.int32, device=dev)
-    with pytest.raises(fa.FAError) as e:
-        fa.backward_varlen(x, x, x, x, x, torch.zeros((2, 10), device=dev), cu, 6)
-    assert e.value.status == fa.FA_ERR_UNSUPPORTED

@@ -49,6 +49,8 @@ CASES = [
     ("mqa d64", 4, 6, 1, 64, False, (100, 300), None),
     ("edges d128", 7, 2, 1, 128, True, None, (1, 0, 128, 129, 256, 0, 37)),
     ("edges d64", 5, 3, 3, 64, False, None, (255, 1, 0, 384, 2)),
+    ("edges d256 causal gqa", 6, 4, 2, 256, True, None, (1, 0, 129, 300, 128, 77)),
+    ("mixed d256", 4, 2, 2, 256, False, (1, 300), None),
 ]
 
 
