@@ -139,3 +139,19 @@ def test_d256_backward_is_bitwise_deterministic():
     _, b = run_fwd_bwd(w, inp)
     for name in ("dq", "dk", "dv"):
         np.testing.assert_array_equal(a[name], b[name], err_msg=name)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_d256_backward_long_sequence_sampled_rows(causal):
+    """B1 H2 N4096 d256: dQ at sampled query rows and dK, dV at sampled key rows of both heads
+    (first, last, 64-query step and 128-key block edges) against the oracle; each dQ row sums
+    the fixed-point contributions of up to 32 key blocks and both feature halves."""
+    w = workloads.custom(1, 2, 4096, 256, causal, seed=8600 + int(causal), std=0.5)
+    inp, got = run_fwd_bwd(w)
+    rows = sorted(set([0, 1, 63, 64, 127, 128, 2047, 2048, 4094, 4095] +
+                      workloads.seeded_sample(8601, 4096, 40)))
+    for h in range(w.H):
+        ref = oracle.head_bwd_rows(inp.q[0, h], inp.k[0, h], inp.v[0, h], inp.do[0, h], rows, rows,
+                                   w.scale, causal)
+        for name in ("dq", "dk", "dv"):
+            assert_grad_close(got[name][0, h, rows], ref[name], name, f"head {h}")
