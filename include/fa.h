@@ -111,6 +111,16 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
                  void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
 /*
+ * fa_selftest_wait_timeout -- a check of the failure path: launches a one-CTA kernel whose
+ * only work is a bounded wait (the same mbarrier wait every kernel of this library uses) on a
+ * barrier that nothing ever completes.  The wait gives up after the current limit
+ * (fa_set_wait_timeout_ns, at least 1 ms) and records FA_ERR_TIMEOUT in the device error flag,
+ * which the next fa_check_device_error returns; the context stays usable.  Nothing faults,
+ * traps or hangs.  Returns FA_OK when launched.
+ */
+FA_API fa_status fa_selftest_wait_timeout(fa_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the calling device's error flag.
  * Returns FA_OK, FA_ERR_INVALID_ARG (a sequence length outside [1, N] was seen),
  * FA_ERR_TIMEOUT (a device-side wait gave up; the outputs of that call are undefined) or

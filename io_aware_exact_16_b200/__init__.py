@@ -61,6 +61,8 @@ _lib.fa_check_device_error.argtypes = [_vp]
 _lib.fa_check_device_error.restype = _i
 _lib.fa_set_kernel_timing_events.argtypes = [_vp, _vp]
 _lib.fa_set_kernel_timing_events.restype = None
+_lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_void_p]
+_lib.fa_selftest_wait_timeout.restype = _i
 _lib.fa_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
 _lib.fa_set_wait_timeout_ns.restype = None
 _lib.fa_status_string.argtypes = [_i]
@@ -70,7 +72,8 @@ _lib.fa_status_string.restype = ctypes.c_char_p
 EXPORTED = ("fa_fwd", "fa_bwd", "fa_fwd_gqa", "fa_bwd_gqa", "fa_fwd_varlen", "fa_bwd_varlen",
             "fa_decode_num_splits", "fa_decode_workspace_size", "fa_fwd_decode",
             "fa_fwd_fp8", "fa_bwd_workspace_size",
-            "fa_check_device_error", "fa_set_wait_timeout_ns", "fa_set_kernel_timing_events",
+            "fa_check_device_error", "fa_selftest_wait_timeout", "fa_set_wait_timeout_ns",
+            "fa_set_kernel_timing_events",
             "fa_status_string",
             "fa_bwd_noalloc")
 
@@ -367,6 +370,16 @@ def check_device_error(device: Optional[torch.device] = None) -> int:
     dev = device or torch.device("cuda", torch.cuda.current_device())
     with torch.cuda.device(dev):
         return int(_lib.fa_check_device_error(_stream_handle(dev)))
+
+
+def selftest_wait_timeout(device: Optional[torch.device] = None) -> None:
+    """``fa_selftest_wait_timeout``: a kernel whose bounded wait can never be satisfied; the next
+    check_device_error() returns FA_ERR_TIMEOUT."""
+    dev = device or torch.device("cuda", torch.cuda.current_device())
+    with torch.cuda.device(dev):
+        st = _lib.fa_selftest_wait_timeout(_stream_handle(dev))
+    if st != FA_OK:
+        raise FAError(st, "fa_selftest_wait_timeout")
 
 
 def set_wait_timeout_ns(ns: int) -> None:

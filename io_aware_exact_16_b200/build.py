@@ -14,7 +14,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 SO = os.path.join(HERE, "libfa.so")
-SOURCES = ["fa_api.cu", "fa_fwd.cu", "fa_bwd.cu", "fa_bwd_noalloc.cu", "fa_bwd_d256.cu", "fa_fwd_d256.cu", "fa_decode.cu",
+SOURCES = ["fa_api.cu", "fa_fwd.cu", "fa_bwd.cu", "fa_bwd_noalloc.cu", "fa_bwd_d256.cu", "fa_fwd_d256.cu", "fa_decode.cu", "fa_selftest.cu",
            "fa_fwd_fp8.cu"]
 HEADERS = ["fa_internal.h", "fa_bwd_common.cuh", "fa_decode.h", "fa_fwd_fp8.h", "sm100.cuh", os.path.join("..", "..", "include", "fa.h")]
 

@@ -262,6 +262,11 @@ fa_status check_decode(int B, int H, int H_kv, int Nq, int N, int d, float scale
 
 using namespace fa;
 
+namespace fa {
+// fa_selftest.cu
+cudaError_t launch_wait_selftest(int* err, uint64_t timeout_ns, cudaStream_t stream);
+}  // namespace fa
+
 extern "C" {
 
 const char* fa_status_string(fa_status s) {
@@ -540,6 +545,16 @@ fa_status fa_fwd_decode(const void* q, const void* k_cache, const void* v_cache,
     take_timing_events(&ev0, &ev1);
     if (launch_decode(d, tq, tk, tv, p, reinterpret_cast<cudaStream_t>(stream), ev0, ev1) !=
         cudaSuccess)
+        return FA_ERR_CUDA;
+    return FA_OK;
+}
+
+fa_status fa_selftest_wait_timeout(fa_stream_t stream) {
+    fa_status st;
+    DeviceState* dev = current_device(&st);
+    if (!dev) return st;
+    if (fa::launch_wait_selftest(dev->err_flag, g_timeout_ns.load(),
+                                 reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
         return FA_ERR_CUDA;
     return FA_OK;
 }

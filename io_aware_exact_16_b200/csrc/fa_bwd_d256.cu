@@ -249,8 +249,8 @@ __global__ void __launch_bounds__(512, 1)
             }
         }
         // Do not leave while our copies may still be landing in shared memory.
-        if (it > 0) mbar_wait(bar_qfull, (it - 1) & 1, p.timeout_ns, abort_flag);
-        mbar_wait(bar_kv, 0, p.timeout_ns, abort_flag);
+        if (it > 0) mbar_wait_drain(bar_qfull, (it - 1) & 1, p.timeout_ns);
+        mbar_wait_drain(bar_kv, 0, p.timeout_ns);
       } else if (warp == 8 && lane == 0) {
         // ------------------------------------------------------------ MMA issuer
         constexpr uint32_t idS = idesc_bf16(128, C::BM, false, false);  // S^T, dP^T
@@ -316,7 +316,7 @@ __global__ void __launch_bounds__(512, 1)
         if (!ok) fail();
         // Wait for every MMA issued here before tensor memory can be released.
         tc_commit(bar_done);
-        mbar_wait(bar_done, 0, p.timeout_ns, abort_flag);
+        mbar_wait_drain(bar_done, 0, p.timeout_ns);
       }
     } else {
         regs_increase<C::REGS_COMPUTE>();

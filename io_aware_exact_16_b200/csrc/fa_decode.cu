@@ -176,8 +176,8 @@ __global__ void __launch_bounds__(192, DecCfg<D>::CTAS_PER_SM)
             if (!ok) fail();
             // Do not leave the CTA while our copies may still be landing in shared memory.
             for (int t = max(0, u - C::NSLOT); t < u; ++t)
-                mbar_wait(&bar_full[t % C::NSLOT], (t / C::NSLOT) & 1, p.timeout_ns, abort_flag);
-            if (!mbar_wait(bar_q, 0, p.timeout_ns, abort_flag)) fail();
+                mbar_wait_drain(&bar_full[t % C::NSLOT], (t / C::NSLOT) & 1, p.timeout_ns);
+            if (!mbar_wait_drain(bar_q, 0, p.timeout_ns)) fail();
         }
     } else if (warp == 4) {
         // ------------------------------------------------------------ MMA issuer
@@ -245,7 +245,7 @@ __global__ void __launch_bounds__(192, DecCfg<D>::CTAS_PER_SM)
             }
             // Wait for every MMA issued here before tensor memory can be released.
             tc_commit(bar_done);
-            mbar_wait(bar_done, 0, p.timeout_ns, abort_flag);
+            mbar_wait_drain(bar_done, 0, p.timeout_ns);
         }
     } else {
         // ------------------------------------------------------------ softmax warpgroup

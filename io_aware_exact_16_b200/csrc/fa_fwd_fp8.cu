@@ -208,10 +208,10 @@ __global__ void __launch_bounds__(384, 1)
             for (int j = max(0, n - C::STAGES); j < n; ++j) {
                 const int s = j % C::STAGES;
                 const uint32_t ph = (j / C::STAGES) & 1;
-                mbar_wait(&bar_kfull[s], ph, p.timeout_ns, abort_flag);
-                mbar_wait(&bar_vfull[s], ph, p.timeout_ns, abort_flag);
+                mbar_wait_drain(&bar_kfull[s], ph, p.timeout_ns);
+                mbar_wait_drain(&bar_vfull[s], ph, p.timeout_ns);
             }
-            if (!mbar_wait(bar_q, 0, p.timeout_ns, abort_flag)) fail();
+            if (!mbar_wait_drain(bar_q, 0, p.timeout_ns)) fail();
         }
       } else if (warp == 8) {
         // ------------------------------------------------------------ MMA issuer
@@ -295,7 +295,7 @@ __global__ void __launch_bounds__(384, 1)
             }
             if (!ok) fail();
             tc_commit(bar_done);
-            mbar_wait(bar_done, 0, p.timeout_ns, abort_flag);
+            mbar_wait_drain(bar_done, 0, p.timeout_ns);
         }
       }
     } else {
