@@ -79,6 +79,42 @@ __device__ __forceinline__ void record_error(int* err, int code) {
     if (err) atomicCAS(err, 0, code);
 }
 
+// Query tile pair cta_x of head (b, h), heaviest causal tiles first.  Causal head-major: the
+// launch order walks groups of up to 16 heads and, within a group, all heads' tiles from the
+// heaviest to the lightest, so the last wave holds light tiles only while one group's K and V
+// (2 N d bf16 per head) stay in L2.  The CTA indices are read with volatile moves so that the
+// epilogue recomputes (b, h) instead of keeping them live through the softmax loop.
+struct CtaCoords {
+    int cta_x, h, b;
+};
+__device__ __forceinline__ CtaCoords cta_coords(bool grouped) {
+    uint32_t bx, by, bz, nx, ny, nz;
+    asm volatile("mov.u32 %0, %%ctaid.x;" : "=r"(bx));
+    asm volatile("mov.u32 %0, %%ctaid.y;" : "=r"(by));
+    asm volatile("mov.u32 %0, %%ctaid.z;" : "=r"(bz));
+    asm volatile("mov.u32 %0, %%nctaid.x;" : "=r"(nx));
+    asm volatile("mov.u32 %0, %%nctaid.y;" : "=r"(ny));
+    asm volatile("mov.u32 %0, %%nctaid.z;" : "=r"(nz));
+    CtaCoords c;
+    if (grouped) {
+        constexpr int GH = 16;
+        const int BH = (int)(ny * nz);
+        const int lin = (int)(bx + nx * (by + ny * bz));
+        const int g0 = lin / ((int)nx * GH) * GH;
+        const int gh = min(GH, BH - g0);     // heads in this group
+        const int r = lin - g0 * (int)nx;    // rank-major position inside the group
+        const int flat = g0 + r % gh;
+        c.cta_x = (int)nx - 1 - r / gh;
+        c.h = flat % (int)ny;
+        c.b = flat / (int)ny;
+    } else {
+        c.cta_x = (int)(nx - 1 - bx);
+        c.h = (int)by;
+        c.b = (int)bz;
+    }
+    return c;
+}
+
 template <int D, bool PACKED>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -90,9 +126,10 @@ __global__ void __launch_bounds__(384, 1)
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    const int cta_x = gridDim.x - 1 - blockIdx.x;  // heaviest (causal) query tiles first
-    const int h = blockIdx.y;
-    const int b = blockIdx.z;
+    const CtaCoords cc = cta_coords(!PACKED && p.causal);
+    const int cta_x = cc.cta_x;
+    const int h = cc.h;
+    const int b = cc.b;
     const int bh = b * p.H + h;
     // Grouped-query attention: consecutive query heads share one key/value head.
     const int h_kv = h / (p.H / p.H_kv);
@@ -409,10 +446,11 @@ __global__ void __launch_bounds__(384, 1)
         if (ok) ok = mbar_wait(&bar_ofull[t], (nt - 1) & 1, p.timeout_ns, abort_flag);
         if (__all_sync(0xffffffffu, ok)) {
             tc_fence_after();
+            const CtaCoords ce = cta_coords(!PACKED && p.causal);  // (b, h) recomputed here
             const float inv_l = l > 0.f ? 1.0f / l : 0.f;
             const bool in_range = row < ext.Lq;
             __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) +
-                                  row_of(packed, b, h, p.H, p.N, ext.t0, in_range ? row : 0) * D;
+                                  row_of(packed, ce.b, ce.h, p.H, p.N, ext.t0, in_range ? row : 0) * D;
 #pragma unroll
             for (int q = 0; q < D / 32; ++q) {
                 uint32_t o[32];
@@ -433,7 +471,7 @@ __global__ void __launch_bounds__(384, 1)
             }
             if (in_range) {
                 // lse in natural-log units: (m + log2 l) * ln 2
-                p.lse[lse_of(packed, b, h, p.H, p.N, p.T, ext.t0, row)] =
+                p.lse[lse_of(packed, ce.b, ce.h, p.H, p.N, p.T, ext.t0, row)] =
                     l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
             }
         } else {
