@@ -99,7 +99,7 @@ struct BwdCfg {
 };
 
 // ---------------------------------------------------------------------------- main kernel
-template <int D, bool PACKED>
+template <int D, bool PACKED, bool GROUPED>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -129,9 +129,24 @@ __global__ void __launch_bounds__(512, 1)
     float* s_scale = reinterpret_cast<float*>(smem + C::SMEM_SCALE);  // [BM]
 
     if (threadIdx.x == 0 && (smem_u32(smem) & 1023u)) record_error(p.err, kErrInvalidArg);
-    const int tile = blockIdx.x;
-    const int bhk = tile / n_kv;  // (batch, key/value head)
-    const int j = tile % n_kv;    // key block (causal: the heaviest, j = 0, first)
+    // Key block j of key/value head bhk.  Head-major causal: the launch order walks groups of
+    // 16 heads and, inside a group, every head's key blocks from the heaviest (j = 0, the most
+    // query blocks) to the lightest, so the last wave holds light blocks only while one
+    // group's Q and dO stay in L2; otherwise head by head, j = 0 first.
+    // (GROUPED: head-major causal launches, their own instantiation.)
+    int bhk, j;
+    if constexpr (GROUPED) {
+        constexpr int GH = 16;
+        const int lin = blockIdx.x;
+        const int g0 = lin / (n_kv * GH) * GH;
+        const int gh = min(GH, (int)(gridDim.x / n_kv) - g0);  // heads in this group
+        const int r = lin - g0 * n_kv;                         // rank-major inside the group
+        bhk = g0 + r % gh;
+        j = r / gh;
+    } else {
+        bhk = blockIdx.x / n_kv;
+        j = blockIdx.x % n_kv;
+    }
     const int b = bhk / p.H_kv;
     const int G = p.H / p.H_kv;   // query heads sharing this key/value head
     const int bh_first = b * p.H + (bhk % p.H_kv) * G;
@@ -611,10 +626,11 @@ cudaError_t launch_bwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
     using C = BwdCfg<D>;
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(fa_bwd_kernel<D, PACKED>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::SMEM_BYTES);
-        if (e != cudaSuccess) return e;
+        for (auto kern : {fa_bwd_kernel<D, PACKED, false>, fa_bwd_kernel<D, PACKED, !PACKED>}) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 C::SMEM_BYTES);
+            if (e != cudaSuccess) return e;
+        }
         configured = true;
     }
     const int BH = p.B * p.H;
@@ -623,7 +639,12 @@ cudaError_t launch_bwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
     const dim3 chunks(p.N_pad / 128, BH);
     fa_bwd_pre_kernel<D><<<chunks, 256, 0, stream>>>(p);
     if (ev_start) cudaEventRecord(ev_start, stream);
-    fa_bwd_kernel<D, PACKED><<<BHkv * n_kv, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
+    // Head-major causal launches take the grouped heaviest-first order (their own
+    // instantiation, so that the other launches keep their code unchanged).
+    if (!PACKED && p.causal)
+        fa_bwd_kernel<D, PACKED, !PACKED><<<BHkv * n_kv, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
+    else
+        fa_bwd_kernel<D, PACKED, false><<<BHkv * n_kv, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
     if (ev_stop) cudaEventRecord(ev_stop, stream);
     fa_bwd_dq_kernel<D><<<chunks, 256, 0, stream>>>(p);
     return cudaGetLastError();

@@ -115,7 +115,7 @@ __device__ __forceinline__ CtaCoords cta_coords(bool grouped) {
     return c;
 }
 
-template <int D, bool PACKED>
+template <int D, bool PACKED, bool GROUPED>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -126,7 +126,11 @@ __global__ void __launch_bounds__(384, 1)
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    const CtaCoords cc = cta_coords(!PACKED && p.causal);
+    // GROUPED (head-major causal launches): the grouped heaviest-first order; otherwise tile
+    // pair gridDim.x - 1 - blockIdx.x (heaviest first) of head (blockIdx.z, blockIdx.y).
+    const CtaCoords cc = GROUPED ? cta_coords(true)
+                                 : CtaCoords{(int)(gridDim.x - 1 - blockIdx.x), (int)blockIdx.y,
+                                             (int)blockIdx.z};
     const int cta_x = cc.cta_x;
     const int h = cc.h;
     const int b = cc.b;
@@ -446,7 +450,7 @@ __global__ void __launch_bounds__(384, 1)
         if (ok) ok = mbar_wait(&bar_ofull[t], (nt - 1) & 1, p.timeout_ns, abort_flag);
         if (__all_sync(0xffffffffu, ok)) {
             tc_fence_after();
-            const CtaCoords ce = cta_coords(!PACKED && p.causal);  // (b, h) recomputed here
+            const CtaCoords ce = GROUPED ? cta_coords(true) : CtaCoords{cta_x, h, b};  // (b, h) recomputed
             const float inv_l = l > 0.f ? 1.0f / l : 0.f;
             const bool in_range = row < ext.Lq;
             __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) +
@@ -494,14 +498,20 @@ cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
     using C = FwdCfg<D>;
     static bool configured = false;  // attribute set once per process (idempotent if raced)
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(fa_fwd_kernel<D, PACKED>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::SMEM_BYTES);
-        if (e != cudaSuccess) return e;
+        for (auto kern : {fa_fwd_kernel<D, PACKED, false>, fa_fwd_kernel<D, PACKED, !PACKED>}) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 C::SMEM_BYTES);
+            if (e != cudaSuccess) return e;
+        }
         configured = true;
     }
     dim3 grid((p.N + C::ROWS_PER_CTA - 1) / C::ROWS_PER_CTA, p.H, B);
-    fa_fwd_kernel<D, PACKED><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    // Head-major causal launches take the grouped heaviest-first order (its own instantiation,
+    // so that the other launches keep their code unchanged).
+    if (!PACKED && p.causal)
+        fa_fwd_kernel<D, PACKED, !PACKED><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    else
+        fa_fwd_kernel<D, PACKED, false><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }
 
