@@ -163,3 +163,13 @@ def test_decode_split_heuristic_and_workspace_size():
                         ((64, 32, 8, 1, 2048, 128), 1), ((8, 32, 8, 4, 8192, 128), 4),
                         ((4, 16, 16, 1, 8192, 256), 2)):
         assert fa.decode_num_splits(*shape) == want, shape
+
+
+def test_wait_selftest_reports_a_missing_device_instead_of_launching():
+    """Host logic only: without a usable sm_100 device the self-test launches nothing and
+    returns an error status (FA_ERR_CUDA or FA_ERR_UNSUPPORTED), as every entry point does."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present; the GPU test covers the launch")
+    st = fa.raw_library().fa_selftest_wait_timeout(None)
+    assert st in (fa.FA_ERR_CUDA, fa.FA_ERR_UNSUPPORTED)
