@@ -19,14 +19,18 @@
 // Deterministic dQ.  Every key block adds a contribution dS_ib K_b to every query row i it
 // sees.  Those contributions are added in integer fixed point, so the sum does not depend on
 // the order in which key blocks arrive and repeated runs are bitwise identical, with no
-// ordering between CTAs.  Row i uses the scale s_i = 2^floor(log2(2^21 / bound_i)), where
+// ordering between CTAs.  Row i uses the scale s_i = 2^floor(log2(2^29 / bound_i)), where
 //     bound_i = 2 |dO_i| max_j |v_j| max_{j,l} |k_jl|
 // bounds every partial sum: sum_j |dS_ij| = sum_j P_ij |dP_ij - D_i| <= 2 |dO_i| max_j |v_j|
 // (|dP_ij| <= |dO_i||v_j|, |D_i| <= |dO_i||O_i| and O_i is a convex combination of the v_j), and
 // each feature of sum_j dS_ij k_j is at most that times max |k_jl|.  Every contribution and
-// every partial sum therefore stays below 2^21 (+ one rounding per key block): far from int32
-// overflow, and below 2^22, where the rounding to an integer can run on the FMA pipe
-// (to_fixed).  Each contribution is rounded once, to 2^-21 bound_i.
+// every partial sum therefore stays below 2^29 (+ one rounding per key block), a factor 4
+// inside int32.  Each contribution is rounded once, to 2^-29 bound_i, exactly to the nearest
+// integer on the FMA and integer pipes (to_fixed).  The bound holds for any inputs, but it is
+// loose (random signs cancel in the sum over keys, which no a-priori bound can use): at
+// N = 16384 the actual dQ uses about 2^-11 of it, so the resolution has to be this fine for
+// the rounding to stay well below the bf16 rounding of dS, also when one value row or one
+// key feature is much larger than the rest.
 //
 // Main-kernel warp roles (512 threads = 4 warpgroups):
 //   warps 0-7   compute: warpgroup h owns query columns [64h, 64h+64) of every block; thread
@@ -167,6 +171,7 @@ __global__ void __launch_bounds__(512, 1)
         if (packed) return;
         // Every key of this block is padding: dK = dV = 0 and no dQ contribution.
         const int rows = min(C::BN, p.N - k0);
+        if (!in_bounds(p.err, ((size_t)bhk * p.N + k0) * D, (size_t)rows * D, p.dbg.kv)) return;
         uint4* dk = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.dk) + ((size_t)bhk * p.N + k0) * D);
         uint4* dv = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.dv) + ((size_t)bhk * p.N + k0) * D);
         for (int i = threadIdx.x; i < rows * D / 8; i += blockDim.x) {
@@ -246,8 +251,10 @@ __global__ void __launch_bounds__(512, 1)
             // warps; barrier 2 before the reads and again after the last read of the step
             {
                 const int q = q0 + r;
-                s_scale[r] =
-                    q < ext.Lq ? fixed_point_scale(p.dOnorm[(size_t)q_head(st) * p.N + q], factor) : 0.f;
+                // (-1, a bound beyond fp32 range, adds nothing; the dQ conversion reports it)
+                s_scale[r] = q < ext.Lq && in_bounds(p.err, (size_t)q_head(st) * p.N + q, 1, p.dbg.vec)
+                                 ? fmaxf(fixed_point_scale(p.dOnorm[(size_t)q_head(st) * p.N + q], factor), 0.f)
+                                 : 0.f;
             }
             named_barrier(2, 128);
             const float* sc = s_scale;
@@ -264,29 +271,40 @@ __global__ void __launch_bounds__(512, 1)
                 tc_fence_before();
                 mbar_arrive(bar_dqempty);           // B may take the next dP^T
                 int* acc = p.dq_acc + ((size_t)q_head(st) * p.N_pad + q0) * D;
-                if constexpr (D == 128) {
-                    // dQ^T: lane = feature r, column = query e; a warp instruction covers 32
-                    // consecutive features of one query row: one 128-byte line.
+                if (in_bounds(p.err, ((size_t)q_head(st) * p.N_pad + q0) * D, (size_t)C::BM * D,
+                              p.dbg.acc)) {
+                    if constexpr (D == 128) {
+                        // dQ^T: lane = feature r, column = query e; a warp instruction covers 32
+                        // consecutive features of one query row: one 128-byte line.
 #pragma unroll
-                    for (int e = 0; e < 128; ++e)
-                        red_add_s32(acc + (size_t)e * D + r, to_fixed(__uint_as_float(v[e]), sc[e]));
-                } else {
-                    // dQ: lane = query r, 64 features.  Convert, transpose 32 x 32 through
-                    // shared memory, then a warp instruction covers 32 consecutive features of
-                    // one row.
-                    int* xp = reinterpret_cast<int*>(smem + C::SMEM_XPOSE) + (warp % 4) * 32 * 33;
-                    const float s_row = sc[r];
+                        for (int e = 0; e < 128; e += 2) {
+                            const int2 x = to_fixed2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                                                     sc[e], sc[e + 1]);
+                            red_add_s32(acc + (size_t)e * D + r, x.x);
+                            red_add_s32(acc + (size_t)(e + 1) * D + r, x.y);
+                        }
+                    } else {
+                        // dQ: lane = query r, 64 features.  Convert, transpose 32 x 32 through
+                        // shared memory, then a warp instruction covers 32 consecutive features of
+                        // one row.
+                        int* xp = reinterpret_cast<int*>(smem + C::SMEM_XPOSE) + (warp % 4) * 32 * 33;
+                        const float s_row = sc[r];
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
+                        for (int c = 0; c < 2; ++c) {
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            xp[lane * 33 + e] = to_fixed(__uint_as_float(v[32 * c + e]), s_row);
-                        __syncwarp();
+                            for (int e = 0; e < 32; e += 2) {
+                                const int2 x = to_fixed2(__uint_as_float(v[32 * c + e]),
+                                                         __uint_as_float(v[32 * c + e + 1]), s_row, s_row);
+                                xp[lane * 33 + e] = x.x;
+                                xp[lane * 33 + e + 1] = x.y;
+                            }
+                            __syncwarp();
 #pragma unroll 4
-                        for (int row = 0; row < 32; ++row)
-                            red_add_s32(acc + (size_t)((warp % 4) * 32 + row) * D + 32 * c + lane,
-                                        xp[row * 33 + lane]);
-                        __syncwarp();
+                            for (int row = 0; row < 32; ++row)
+                                red_add_s32(acc + (size_t)((warp % 4) * 32 + row) * D + 32 * c + lane,
+                                            xp[row * 33 + lane]);
+                            __syncwarp();
+                        }
                     }
                 }
             }
@@ -462,9 +480,11 @@ __global__ void __launch_bounds__(512, 1)
         auto load_vectors = [&](Step st) {
             const int q = q_block(st) * C::BM + (ct & 127);
             if (ct < 128)
-                staged = q < ext.Lq ? -p.lse[lse_base + (size_t)st.g * lse_hstride + q] * kLog2e
-                                    : -INFINITY;
-            else staged = q < ext.Lq ? p.Dvec[(size_t)q_head(st) * p.N + q] : 0.f;
+                staged = q < ext.Lq && in_bounds(p.err, lse_base + (size_t)st.g * lse_hstride + q, 1, p.dbg.lse)
+                             ? -p.lse[lse_base + (size_t)st.g * lse_hstride + q] * kLog2e
+                             : -INFINITY;
+            else staged = q < ext.Lq && in_bounds(p.err, (size_t)q_head(st) * p.N + q, 1, p.dbg.vec)
+                             ? p.Dvec[(size_t)q_head(st) * p.N + q] : 0.f;
         };
         auto store_vectors = [&](int it) {
             if (ct < 128) s_lse2[(it & 1) * C::BM + ct] = staged;
@@ -581,11 +601,12 @@ __global__ void __launch_bounds__(512, 1)
         if (ok) ok = mbar_wait(bar_done, 0, p.timeout_ns, abort_flag);  // every MMA finished
         if (__all_sync(0xffffffffu, ok)) {
             tc_fence_after();
-            const bool in_range = kidx < (packed ? L : p.N);
+            const bool key_row = kidx < (packed ? L : p.N);
             const size_t off =
-                row_of(packed, b, bhk % p.H_kv, p.H_kv, p.N, ext.t0, in_range ? kidx : 0) * D;
+                row_of(packed, b, bhk % p.H_kv, p.H_kv, p.N, ext.t0, key_row ? kidx : 0) * D;
             const uint32_t col0 = h ? C::TM_DK : C::TM_DV;
             const float mul = h ? p.scale : 1.0f;
+            const bool in_range = key_row && in_bounds(p.err, off, D, p.dbg.kv);
             __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(h ? p.dk : p.dv) + off;
 #pragma unroll
             for (int q = 0; q < D / 32; ++q) {
@@ -624,15 +645,12 @@ cudaError_t launch_bwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
                          const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream,
                          cudaEvent_t ev_start, cudaEvent_t ev_stop) {
     using C = BwdCfg<D>;
-    static bool configured = false;
-    if (!configured) {
-        for (auto kern : {fa_bwd_kernel<D, PACKED, false>, fa_bwd_kernel<D, PACKED, !PACKED>}) {
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 C::SMEM_BYTES);
-            if (e != cudaSuccess) return e;
-        }
-        configured = true;
-    }
+    static std::atomic<uint64_t> configured{0};  // one bit per device
+    if (cudaError_t e = set_smem_limit_once(configured, C::SMEM_BYTES,
+                                            fa_bwd_kernel<D, PACKED, false>,
+                                            fa_bwd_kernel<D, PACKED, !PACKED>);
+        e != cudaSuccess)
+        return e;
     const int BH = p.B * p.H;
     const int n_kv = (p.N + C::BN - 1) / C::BN;
     const int BHkv = p.B * p.H_kv;

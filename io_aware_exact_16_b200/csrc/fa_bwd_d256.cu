@@ -128,6 +128,7 @@ __global__ void __launch_bounds__(512, 1)
         if (packed) return;
         // Every key of this block is padding: dK = dV = 0 (this CTA's feature half).
         const int rows = min(C::BN, p.N - k0);
+        if (!in_bounds(p.err, ((size_t)bhk * p.N + k0) * D, (size_t)rows * D, p.dbg.kv)) return;
         __nv_bfloat16* dk = reinterpret_cast<__nv_bfloat16*>(p.dk) + ((size_t)bhk * p.N + k0) * D;
         __nv_bfloat16* dv = reinterpret_cast<__nv_bfloat16*>(p.dv) + ((size_t)bhk * p.N + k0) * D;
         for (int i = threadIdx.x; i < rows * (C::DH / 8); i += blockDim.x) {
@@ -195,8 +196,9 @@ __global__ void __launch_bounds__(512, 1)
             const int q0 = q_block(st) * C::BM;
             if (r < C::BM) {  // fixed-point scale of query q0 + r (rows past N: 0)
                 const int q = q0 + r;
-                s_scale[r] =
-                    q < ext.Lq ? fixed_point_scale(p.dOnorm[(size_t)q_head(st) * p.N + q], factor) : 0.f;
+                s_scale[r] = q < ext.Lq && in_bounds(p.err, (size_t)q_head(st) * p.N + q, 1, p.dbg.vec)
+                                 ? fmaxf(fixed_point_scale(p.dOnorm[(size_t)q_head(st) * p.N + q], factor), 0.f)
+                                 : 0.f;
             }
             named_barrier(2, 128);
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_dqfull, it & 1, p.timeout_ns, abort_flag));
@@ -213,9 +215,17 @@ __global__ void __launch_bounds__(512, 1)
                 // dQ^T: lane = feature, column = query e: a warp instruction covers 32
                 // consecutive features of one query row, one 128-byte line.
                 int* acc = p.dq_acc + ((size_t)q_head(st) * p.N_pad + q0) * D + hd * C::DH + r;
+                const bool acc_ok = in_bounds(p.err, ((size_t)q_head(st) * p.N_pad + q0) * D,
+                                              (size_t)C::BM * D, p.dbg.acc);
+                if (acc_ok) {
 #pragma unroll
-                for (int e = 0; e < C::BM; ++e)
-                    red_add_s32(acc + (size_t)e * D, to_fixed(__uint_as_float(v[e]), s_scale[e]));
+                    for (int e = 0; e < C::BM; e += 2) {
+                        const int2 x = to_fixed2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                                                 s_scale[e], s_scale[e + 1]);
+                        red_add_s32(acc + (size_t)e * D, x.x);
+                        red_add_s32(acc + (size_t)(e + 1) * D, x.y);
+                    }
+                }
             }
             named_barrier(2, 128);  // every read of s_scale done before the next step writes
         }
@@ -341,10 +351,12 @@ __global__ void __launch_bounds__(512, 1)
         auto load_vectors = [&](Step s) {
             const int q = q_block(s) * C::BM + (ct & 63);
             if (ct < 64)
-                staged = q < ext.Lq ? -p.lse[lse_base + (size_t)s.g * lse_hstride + q] * kLog2e
-                                    : -INFINITY;
+                staged = q < ext.Lq && in_bounds(p.err, lse_base + (size_t)s.g * lse_hstride + q, 1, p.dbg.lse)
+                             ? -p.lse[lse_base + (size_t)s.g * lse_hstride + q] * kLog2e
+                             : -INFINITY;
             else if (ct < 128)
-                staged = q < ext.Lq ? p.Dvec[(size_t)q_head(s) * p.N + q] : 0.f;
+                staged = q < ext.Lq && in_bounds(p.err, (size_t)q_head(s) * p.N + q, 1, p.dbg.vec)
+                             ? p.Dvec[(size_t)q_head(s) * p.N + q] : 0.f;
         };
         auto store_vectors = [&](int it) {
             if (ct < 64) s_lse2[(it & 1) * C::BM + ct] = staged;
@@ -453,12 +465,13 @@ __global__ void __launch_bounds__(512, 1)
         if (ok) ok = mbar_wait(bar_done, 0, p.timeout_ns, abort_flag);  // every MMA finished
         if (__all_sync(0xffffffffu, ok)) {
             tc_fence_after();
-            const bool in_range = kidx < (packed ? L : p.N);
+            const bool key_row = kidx < (packed ? L : p.N);
             const size_t off =
-                row_of(packed, b, bhk % p.H_kv, p.H_kv, p.N, ext.t0, in_range ? kidx : 0) * D +
+                row_of(packed, b, bhk % p.H_kv, p.H_kv, p.N, ext.t0, key_row ? kidx : 0) * D +
                 hd * C::DH;
             const uint32_t col0 = h ? C::TM_DK : C::TM_DV;
             const float mul = h ? p.scale : 1.0f;
+            const bool in_range = key_row && in_bounds(p.err, off, C::DH, p.dbg.kv);
             __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(h ? p.dk : p.dv) + off;
 #pragma unroll 1
             for (int q = 0; q < C::DH / 32; ++q) {
@@ -498,15 +511,11 @@ cudaError_t launch_bwd_d256(const CUtensorMap& tq, const CUtensorMap& tk, const 
                             const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream,
                             cudaEvent_t ev_start, cudaEvent_t ev_stop) {
     using C = Bwd256;
-    static bool configured = false;  // attribute set once per process (idempotent if raced)
-    if (!configured) {
-        for (auto kern : {fa_bwd_d256_kernel<false>, fa_bwd_d256_kernel<true>}) {
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 C::SMEM_BYTES);
-            if (e != cudaSuccess) return e;
-        }
-        configured = true;
-    }
+    static std::atomic<uint64_t> configured{0};  // one bit per device
+    if (cudaError_t e = set_smem_limit_once(configured, C::SMEM_BYTES,
+                                            fa_bwd_d256_kernel<false>, fa_bwd_d256_kernel<true>);
+        e != cudaSuccess)
+        return e;
     const dim3 chunks(p.N_pad / 128, p.B * p.H);
     const int n_kv = (p.N + C::BN - 1) / C::BN;
     fa_bwd_pre_kernel<256><<<chunks, 256, 0, stream>>>(p);

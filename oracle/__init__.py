@@ -174,6 +174,37 @@ def head_bwd_rows(q, k, v, do, qrows: Sequence[int], krows: Sequence[int], scale
     return {"dq": dq[:len(qr)], "dk": dk[:len(kr)], "dv": dv[:len(kr)]}
 
 
+def dq_magnitude_sums(q, k, v, do, rows: Sequence[int], scale: float, causal: bool):
+    """Magnitudes that bound how far a dQ formed from rounded operands can be from the exact
+    one, for the listed query rows of one head (fp64 numpy, no blocking):
+
+      abs_dS_k[r, l] = sum_j |dS_ij| |k_jl|                  (rounding each dS_ij moves dQ_il
+                                                               by at most its share of this)
+      D_term[r, l]   = |dO_i| |O_i| sum_j P_ij |k_jl|         (rounding O moves D_i, and with
+                                                               it every dS_ij, by P_ij dD_i)
+
+    with i = rows[r] and the definitions of the backward pass: s_ij = scale q_i . k_j over the
+    visible keys j (j <= i when causal), P_ij = exp(s_ij - lse_i), O_i = sum_j P_ij v_j,
+    dP_ij = dO_i . v_j, D_i = dO_i . O_i, dS_ij = P_ij (dP_ij - D_i).  dQ_il = scale sum_j
+    dS_ij k_jl, so |dQ_il| <= scale abs_dS_k[r, l].  Used by tolerances only."""
+    q, k, v, do = as_f64(q), as_f64(k), as_f64(v), as_f64(do)
+    N, d = q.shape
+    absk = np.abs(k)
+    A = np.zeros((len(rows), d), np.float64)
+    Dt = np.zeros((len(rows), d), np.float64)
+    for r, i in enumerate(rows):
+        lim = i + 1 if causal else N
+        s_row = scale * (k[:lim] @ q[i])
+        e = np.exp(s_row - s_row.max())
+        P = e / e.sum()
+        O = P @ v[:lim]
+        dP = v[:lim] @ do[i]
+        dS = P * (dP - do[i] @ O)
+        A[r] = np.abs(dS) @ absk[:lim]
+        Dt[r] = np.linalg.norm(do[i]) * np.linalg.norm(O) * (P @ absk[:lim])
+    return {"abs_dS_k": A, "D_term": Dt}
+
+
 def _lengths(seqlens, B: int, N: int) -> list[int]:
     if seqlens is None:
         return [N] * B

@@ -48,6 +48,10 @@ SMALL = [
     (4, 2, 333, 64, True, (1, 333)),
     (2, 2, 512, 64, False, (128, 512)),
     (2, 1, 520, 128, True, (100, 520)),
+    # causal launches walk groups of 16 heads: B*H = 21 is one full group and a partial one
+    (3, 7, 300, 128, True, None),
+    (3, 7, 300, 64, True, None),
+    (3, 7, 300, 64, True, (70, 300)),
 ]
 
 
@@ -88,17 +92,3 @@ def test_padded_keys_get_zero_gradient_and_garbage_changes_nothing():
     _, b = run_fwd_bwd(w, workloads.Inputs(inp.q, k2, v2, inp.do, inp.seqlens))
     for name in ("o", "lse", "dq", "dk", "dv"):
         np.testing.assert_array_equal(a[name], b[name], err_msg=name)
-
-
-@pytest.mark.parametrize("HD,causal", [((16, 128), False), ((16, 128), True), ((32, 64), False)])
-def test_sweep_N4096_sampled_heads(HD, causal):
-    """Throughput-sweep shape at N = 4096: 2 seeded heads checked in full."""
-    H, d = HD
-    w = workloads.sweep(4096, H, d, causal)
-    inp, got = run_fwd_bwd(w)
-    for flat in workloads.seeded_sample(w.seed, w.B * w.H, 2):
-        b, h = divmod(flat, w.H)
-        ref = oracle.head_bwd(inp.q[b, h], inp.k[b, h], inp.v[b, h], inp.do[b, h], w.scale, causal)
-        assert_fwd_close(got["o"][b, h], got["lse"][b, h], ref["o"], ref["lse"], f"{w.name} b{b}h{h}")
-        for name in ("dq", "dk", "dv"):
-            assert_grad_close(got[name][b, h], ref[name], name, f"{w.name} b{b}h{h}")

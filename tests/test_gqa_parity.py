@@ -32,6 +32,9 @@ SHAPES = [
     (3, 4, 2, 384, 128, False, (1, 384)),
     (2, 4, 1, 200, 64, True, (50, 200)),
     (2, 12, 4, 1024, 64, True, None),       # GPT-2-small shape with 4 key/value heads
+    # causal launches walk groups of 16 heads: B*H_kv = 21 is one full group and a partial one
+    (3, 14, 7, 300, 128, True, None),
+    (3, 14, 7, 300, 64, True, None),
 ]
 
 

@@ -589,3 +589,42 @@ def test_fp8_attention_is_attention_of_the_dequantised_values():
     assert np.abs(2.0 * O - O2).max() < 1e-12 and np.abs(lse - lse2).max() == 0.0
     # the quantised values stay within one e4m3 step (2^-3 relative) of the fp32 draws
     assert np.all(np.abs(f.q.float().abs().numpy()) <= 448.0)
+
+
+# ---------------------------------------------------------------- dQ rounding magnitudes
+@pytest.mark.parametrize("causal", [False, True])
+def test_dq_magnitude_sums_bound_dq_and_match_brute_force(causal):
+    """oracle.dq_magnitude_sums (used by the tolerances of the fixed-point dQ tests): checked
+    against explicit loops over keys written here from the definitions (softmax of the scaled
+    scores over the visible keys, dS = P (dP - D), D = dO . O), against the C oracle's dQ
+    (|dQ_il| <= scale * sum_j |dS_ij| |k_jl|, the triangle inequality), and on special cases
+    (one visible key: dS = 0, so the first sum vanishes; Q = 0: P is uniform, so the second
+    sum is |dO| |O| times the mean of |k|)."""
+    N, d, scale = 9, 4, 0.37
+    q, k, v, do = (bf16_head(N, d, 900 + i) for i in range(4))
+    rows = [0, 3, 8]
+    got = oracle.dq_magnitude_sums(q, k, v, do, rows, scale, causal)
+    for r, i in enumerate(rows):
+        J = [j for j in range(N) if visible(i, j, N, causal)]
+        s = [scale * sum(q[i, c] * k[j, c] for c in range(d)) for j in J]
+        m = max(s)
+        z = sum(math.exp(x - m) for x in s)
+        P = [math.exp(x - m) / z for x in s]
+        O = [sum(P[t] * v[j, c] for t, j in enumerate(J)) for c in range(d)]
+        D = sum(do[i, c] * O[c] for c in range(d))
+        dS = [P[t] * (sum(do[i, c] * v[j, c] for c in range(d)) - D) for t, j in enumerate(J)]
+        no = math.sqrt(sum(x * x for x in do[i])) * math.sqrt(sum(x * x for x in O))
+        for c in range(d):
+            a = sum(abs(dS[t]) * abs(k[j, c]) for t, j in enumerate(J))
+            b = no * sum(P[t] * abs(k[j, c]) for t, j in enumerate(J))
+            assert abs(got["abs_dS_k"][r, c] - a) <= 1e-12 * max(1.0, a)
+            assert abs(got["D_term"][r, c] - b) <= 1e-12 * max(1.0, b)
+    ref = oracle.head_bwd(q, k, v, do, scale, causal)
+    bound = oracle.dq_magnitude_sums(q, k, v, do, list(range(N)), scale, causal)
+    assert np.all(np.abs(ref["dq"]) <= scale * bound["abs_dS_k"] * (1 + 1e-12) + 1e-15)
+    if causal:
+        assert np.all(bound["abs_dS_k"][0] == 0)  # row 0 sees one key
+    z = oracle.dq_magnitude_sums(np.zeros_like(q), k, v, do, [N - 1], scale, False)
+    O = v.mean(0)
+    want = np.linalg.norm(do[N - 1]) * np.linalg.norm(O) * np.abs(k).mean(0)
+    assert np.allclose(z["D_term"][0], want, rtol=1e-12, atol=0)
