@@ -101,9 +101,11 @@ FA_API size_t fa_bwd_workspace_size(int B, int H, int N, int d);
  *   workspace      scratch of at least fa_bwd_workspace_size(B, H, N, d) bytes, 16-byte
  *                  aligned, owned by the caller, not used concurrently by another call.
  * The dQ sum over key blocks is exact integer (fixed-point) arithmetic: each key block's
- * contribution to query row i is rounded once to 2^-21 of an a-priori bound of row i
+ * contribution to query row i is rounded once to 2^-29 of an a-priori bound of row i
  * (2 |dO_i| max_j |v_j| max |k|) and the integer sum does not depend on the order in which
  * key blocks arrive, so repeated calls on the same inputs give bitwise identical dq, dk, dv.
+ * Inputs so large that this bound is not finite in fp32 (norms beyond 3.4e38) leave that
+ * row's dq at 0 and record FA_ERR_INVALID_ARG in the device error flag.
  */
 FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
                  const float* lse, void* dq, void* dk, void* dv,
@@ -121,8 +123,25 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
 FA_API fa_status fa_selftest_wait_timeout(fa_stream_t stream);
 
 /*
+ * Index checks.  The library also comes as a checking build (libfa_debug.so, the same sources
+ * compiled with FA_DEBUG), a stand-in for a memory sanitizer: in it every plain load and store
+ * of global memory in the kernels (the accesses not made by TMA, whose tensor maps bound them)
+ * first checks its index against the buffer it belongs to; an index outside records
+ * FA_ERR_INVALID_ARG in the device error flag and the access is skipped.  Nothing traps.
+ * fa_debug_checks returns 1 in that build and 0 in the release build.
+ *
+ * fa_selftest_bounds exercises that check: one thread stores `value` to buf[n - 1] and to
+ * buf[n] (one past a caller-owned device buffer of n >= 1 ints, 4-byte aligned) through it, so
+ * buf[n - 1] is written, buf[n] is not, and the next fa_check_device_error returns
+ * FA_ERR_INVALID_ARG.  The release build returns FA_ERR_UNSUPPORTED and launches nothing.
+ */
+FA_API int fa_debug_checks(void);
+FA_API fa_status fa_selftest_bounds(int* buf, int n, int value, fa_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the calling device's error flag.
- * Returns FA_OK, FA_ERR_INVALID_ARG (a sequence length outside [1, N] was seen),
+ * Returns FA_OK, FA_ERR_INVALID_ARG (a sequence length outside [1, N] was seen, or a
+ * backward row whose fixed-point bound overflowed fp32),
  * FA_ERR_TIMEOUT (a device-side wait gave up; the outputs of that call are undefined) or
  * FA_ERR_CUDA (the synchronisation itself failed).
  */
@@ -253,22 +272,29 @@ FA_API fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, const f
  *
  * It computes exactly what fa_bwd computes, with the same kernels, arguments, layouts and
  * results, but its scratch (the workspace fa_bwd takes from the caller) is a fixed area of
- * FA_BWD_NOALLOC_SCRATCH_BYTES inside this library's own device code image: every GPU that
- * loads the library holds that area until the process exits.  The caller still provides
+ * FA_BWD_NOALLOC_SCRATCH_BYTES inside this library's own device code image: every GPU on which
+ * that image is loaded holds the area until the process exits.  The caller still provides
  * every input and output buffer.
  *   error_flag  optional caller-owned device int (4-byte aligned): device-side errors of this
  *               call (a bad sequence length, a wait that timed out) are stored there as an
  *               fa_status code; it is never cleared by the library.  NULL: not reported.
  * Limits and rules:
  *   - Problems whose fa_bwd_workspace_size(B, H, N, d) exceeds FA_BWD_NOALLOC_SCRATCH_BYTES
- *     are rejected with FA_ERR_WORKSPACE (e.g. B*H = 16, N = 4096, d = 128 fits;
- *     B*H = 64 at the same N and d does not).
+ *     are rejected with FA_ERR_WORKSPACE (e.g. B*H = 31, N = 4096, d = 128 fits;
+ *     B*H = 32 at the same N and d does not).
  *   - All calls on a device share the one scratch area and each call overwrites it.  Calls
  *     whose kernels overlap on the GPU (other streams, other host threads) race and give
  *     wrong results: issue them on one stream, or order them yourself.
  *   - The first call on a device performs a one-time set-up on the host (it looks up the
  *     scratch area's device address); make that first call before any stream capture.
- *   - No cudaMalloc, cudaFree or other allocating call is made, ever.
+ *   - When the area is placed in device memory depends on CUDA's module loading.  Under lazy
+ *     loading (the default since CUDA 12.2) it is placed by that first call on each device,
+ *     not when the library is loaded: a caller that reserves the rest of the device memory for
+ *     its own pool should make the first call before reserving it (or run with
+ *     CUDA_MODULE_LOADING=EAGER, which places the area when the library's code is loaded).  If
+ *     the first call finds no room for the area it returns FA_ERR_WORKSPACE and launches
+ *     nothing; a later call tries again.
+ *   - No cudaMalloc, cudaFree or other allocating call is made by this entry point.
  */
 #define FA_BWD_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 FA_API fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,

@@ -28,51 +28,64 @@ except OSError as exc:  # pragma: no cover
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
-_lib.fa_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, ctypes.c_float, _i, _vp, _vp]
-_lib.fa_fwd.restype = _i
-_lib.fa_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
-                        ctypes.c_float, _i, _vp, _vp, ctypes.c_size_t, _vp]
-_lib.fa_bwd.restype = _i
-_lib.fa_fwd_gqa.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float, _i, _vp,
-                            _vp]
-_lib.fa_fwd_gqa.restype = _i
-_lib.fa_bwd_gqa.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
-                            ctypes.c_float, _i, _vp, _vp, ctypes.c_size_t, _vp]
-_lib.fa_bwd_gqa.restype = _i
-_lib.fa_fwd_varlen.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
-                               ctypes.c_float, _i, _vp]
-_lib.fa_fwd_varlen.restype = _i
-_lib.fa_bwd_varlen.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
-                               _i, _i, ctypes.c_float, _i, _vp, ctypes.c_size_t, _vp]
-_lib.fa_bwd_varlen.restype = _i
-_lib.fa_decode_num_splits.argtypes = [_i, _i, _i, _i, _i, _i, _i]
-_lib.fa_decode_num_splits.restype = _i
-_lib.fa_decode_workspace_size.argtypes = [_i, _i, _i, _i, _i]
-_lib.fa_decode_workspace_size.restype = ctypes.c_size_t
-_lib.fa_fwd_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
-                               ctypes.c_float, _i, _i, _vp, ctypes.c_size_t, _vp]
-_lib.fa_fwd_decode.restype = _i
-_lib.fa_fwd_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
-                            ctypes.c_float, _i, _vp, _vp]
-_lib.fa_fwd_fp8.restype = _i
-_lib.fa_bwd_workspace_size.argtypes = [_i, _i, _i, _i]
-_lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
-_lib.fa_check_device_error.argtypes = [_vp]
-_lib.fa_check_device_error.restype = _i
-_lib.fa_set_kernel_timing_events.argtypes = [_vp, _vp]
-_lib.fa_set_kernel_timing_events.restype = None
-_lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_void_p]
-_lib.fa_selftest_wait_timeout.restype = _i
-_lib.fa_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
-_lib.fa_set_wait_timeout_ns.restype = None
-_lib.fa_status_string.argtypes = [_i]
-_lib.fa_status_string.restype = ctypes.c_char_p
+
+
+def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
+    """Declares the C signatures of include/fa.h on a loaded library handle."""
+    lib.fa_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, ctypes.c_float, _i, _vp, _vp]
+    lib.fa_fwd.restype = _i
+    lib.fa_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                           ctypes.c_float, _i, _vp, _vp, ctypes.c_size_t, _vp]
+    lib.fa_bwd.restype = _i
+    lib.fa_fwd_gqa.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float, _i, _vp,
+                               _vp]
+    lib.fa_fwd_gqa.restype = _i
+    lib.fa_bwd_gqa.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
+                               ctypes.c_float, _i, _vp, _vp, ctypes.c_size_t, _vp]
+    lib.fa_bwd_gqa.restype = _i
+    lib.fa_fwd_varlen.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                                  ctypes.c_float, _i, _vp]
+    lib.fa_fwd_varlen.restype = _i
+    lib.fa_bwd_varlen.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                                  _i, _i, ctypes.c_float, _i, _vp, ctypes.c_size_t, _vp]
+    lib.fa_bwd_varlen.restype = _i
+    lib.fa_decode_num_splits.argtypes = [_i, _i, _i, _i, _i, _i, _i]
+    lib.fa_decode_num_splits.restype = _i
+    lib.fa_decode_workspace_size.argtypes = [_i, _i, _i, _i, _i]
+    lib.fa_decode_workspace_size.restype = ctypes.c_size_t
+    lib.fa_fwd_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                                  ctypes.c_float, _i, _i, _vp, ctypes.c_size_t, _vp]
+    lib.fa_fwd_decode.restype = _i
+    lib.fa_fwd_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
+                               ctypes.c_float, _i, _vp, _vp]
+    lib.fa_fwd_fp8.restype = _i
+    lib.fa_bwd_workspace_size.argtypes = [_i, _i, _i, _i]
+    lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.fa_check_device_error.argtypes = [_vp]
+    lib.fa_check_device_error.restype = _i
+    lib.fa_set_kernel_timing_events.argtypes = [_vp, _vp]
+    lib.fa_set_kernel_timing_events.restype = None
+    lib.fa_selftest_bounds.argtypes = [_vp, _i, _i, _vp]
+    lib.fa_selftest_bounds.restype = _i
+    lib.fa_debug_checks.argtypes = []
+    lib.fa_debug_checks.restype = _i
+    lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_void_p]
+    lib.fa_selftest_wait_timeout.restype = _i
+    lib.fa_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+    lib.fa_set_wait_timeout_ns.restype = None
+    lib.fa_status_string.argtypes = [_i]
+    lib.fa_status_string.restype = ctypes.c_char_p
+    return lib
+
+
+_bind(_lib)
 
 # Every symbol include/fa.h declares.
 EXPORTED = ("fa_fwd", "fa_bwd", "fa_fwd_gqa", "fa_bwd_gqa", "fa_fwd_varlen", "fa_bwd_varlen",
             "fa_decode_num_splits", "fa_decode_workspace_size", "fa_fwd_decode",
             "fa_fwd_fp8", "fa_bwd_workspace_size",
-            "fa_check_device_error", "fa_selftest_wait_timeout", "fa_set_wait_timeout_ns",
+            "fa_check_device_error", "fa_selftest_wait_timeout", "fa_selftest_bounds",
+            "fa_debug_checks", "fa_set_wait_timeout_ns",
             "fa_set_kernel_timing_events",
             "fa_status_string",
             "fa_bwd_noalloc")
@@ -398,3 +411,38 @@ def time_next_kernel(start: "torch.cuda.Event", stop: "torch.cuda.Event") -> Non
 def raw_library() -> ctypes.CDLL:
     """The loaded ctypes handle of ``libfa.so`` (for direct C-ABI calls)."""
     return _lib
+
+
+LIB_DEBUG_PATH = os.path.join(_HERE, "libfa_debug.so")
+_debug_lib: Optional[ctypes.CDLL] = None
+
+
+def debug_library() -> ctypes.CDLL:
+    """The checking build ``libfa_debug.so`` (same C ABI; every plain global load and store in
+    its kernels checks its index against its buffer first, records FA_ERR_INVALID_ARG and skips
+    the access when out of range).  Loaded on first use; raises ImportError if it is missing."""
+    global _debug_lib
+    if _debug_lib is None:
+        if not os.path.exists(LIB_DEBUG_PATH):
+            raise ImportError(f"{LIB_DEBUG_PATH} is missing: build it with "
+                              "`python io_aware_exact_16_b200/build.py`")
+        _debug_lib = _bind(ctypes.CDLL(LIB_DEBUG_PATH))
+    return _debug_lib
+
+
+class use_library:
+    """Context manager: the functions of this module call `lib` (e.g. debug_library()) instead
+    of libfa.so inside the block.  Not thread-safe; meant for tests."""
+
+    def __init__(self, lib: ctypes.CDLL):
+        self.lib = lib
+
+    def __enter__(self):
+        global _lib
+        self.saved, _lib = _lib, self.lib
+        return self.lib
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self.saved
+

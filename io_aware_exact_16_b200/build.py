@@ -1,4 +1,7 @@
-"""Builds the CUDA library ``libfa.so`` in-tree for sm_100a with nvcc.
+"""Builds the CUDA library ``libfa.so`` in-tree for sm_100a with nvcc, and its checking twin
+``libfa_debug.so`` (the same sources compiled with FA_DEBUG: every plain global load and store
+in the kernels checks its index against the buffer it belongs to, records FA_ERR_INVALID_ARG
+and skips the access when it is out of range; nothing traps).
 
 The library is the C ABI of ``include/fa.h``; the Python binding in this package loads it
 with ctypes.  Run ``python io_aware_exact_16_b200/build.py`` (a plain script: importing the
@@ -14,6 +17,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 SO = os.path.join(HERE, "libfa.so")
+SO_DEBUG = os.path.join(HERE, "libfa_debug.so")
 SOURCES = ["fa_api.cu", "fa_fwd.cu", "fa_bwd.cu", "fa_bwd_noalloc.cu", "fa_bwd_d256.cu", "fa_fwd_d256.cu", "fa_decode.cu", "fa_selftest.cu",
            "fa_fwd_fp8.cu"]
 HEADERS = ["fa_internal.h", "fa_bwd_common.cuh", "fa_decode.h", "fa_fwd_fp8.h", "sm100.cuh", os.path.join("..", "..", "include", "fa.h")]
@@ -34,39 +38,46 @@ def flags() -> list[str]:
             "-Xptxas", "-v", "--expt-relaxed-constexpr"]
 
 
-def _stale() -> bool:
-    if not os.path.exists(SO):
+def _stale(so: str) -> bool:
+    if not os.path.exists(so):
         return True
-    t = os.path.getmtime(SO)
+    t = os.path.getmtime(so)
     for f in SOURCES + HEADERS:
         if os.path.getmtime(os.path.join(CSRC, f)) > t:
             return True
     return False
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
-        return SO
+def _build_one(so: str, extra: list[str], build_dir: str, verbose: bool) -> str:
     objs = []
-    build_dir = os.path.join(HERE, "_build")
     os.makedirs(build_dir, exist_ok=True)
     for src in SOURCES:
         obj = os.path.join(build_dir, src.replace(".cu", ".o"))
-        cmd = [nvcc(), *flags(), "-c", os.path.join(CSRC, src), "-o", obj]
+        cmd = [nvcc(), *flags(), *extra, "-c", os.path.join(CSRC, src), "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if verbose or r.returncode != 0:
             sys.stderr.write(r.stdout + r.stderr)
         if r.returncode != 0:
             raise RuntimeError(f"nvcc failed on {src}")
         objs.append(obj)
-    tmp = SO + ".tmp"
+    tmp = so + ".tmp"
     cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs,
            "-Xcompiler", "-fPIC"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         sys.stderr.write(r.stdout + r.stderr)
         raise RuntimeError("nvcc link failed")
-    os.replace(tmp, SO)
+    os.replace(tmp, so)
+    return so
+
+
+def build(force: bool = False, verbose: bool = False, debug: bool = True) -> str:
+    """Builds libfa.so (and, unless debug=False, libfa_debug.so); returns libfa.so's path."""
+    build_dir = os.path.join(HERE, "_build")
+    if force or _stale(SO):
+        _build_one(SO, [], build_dir, verbose)
+    if debug and (force or _stale(SO_DEBUG)):
+        _build_one(SO_DEBUG, ["-DFA_DEBUG"], os.path.join(build_dir, "debug"), verbose)
     return SO
 
 

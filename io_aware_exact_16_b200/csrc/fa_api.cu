@@ -205,6 +205,7 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
     p.timeout_ns = g_timeout_ns.load();
+    p.dbg = extents(B, H, H_kv, N, d, T, packed);
     cudaEvent_t ev0, ev1;
     take_timing_events(&ev0, &ev1);
     if (ev0) cudaEventRecord(ev0, stream);
@@ -265,6 +266,7 @@ using namespace fa;
 namespace fa {
 // fa_selftest.cu
 cudaError_t launch_wait_selftest(int* err, uint64_t timeout_ns, cudaStream_t stream);
+cudaError_t launch_bounds_selftest(int* buf, int n, int value, int* err, cudaStream_t stream);
 }  // namespace fa
 
 extern "C" {
@@ -374,8 +376,9 @@ static fa_status bwd_impl(const void* q, const void* k, const void* v, const voi
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
     p.timeout_ns = g_timeout_ns.load();
-
     const bool packed = cu_seqlens != nullptr;
+    p.dbg = extents(B, H, H_kv, N, d, T, packed);
+
     CUtensorMap tq, tk, tv, tdo;
     const int q_rows = d == 256 ? 64 : 128;  // query rows per backward step
     if (!user_map(&tq, q, d, B, H, N, T, packed, q_rows) ||
@@ -451,6 +454,7 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, const float* q
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
     p.timeout_ns = g_timeout_ns.load();
+    p.dbg = extents(B, H, H_kv, N, d, 0, false);
     cudaEvent_t ev0, ev1;
     take_timing_events(&ev0, &ev1);
     const cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
@@ -535,6 +539,12 @@ fa_status fa_fwd_decode(const void* q, const void* k_cache, const void* v_cache,
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
     p.timeout_ns = g_timeout_ns.load();
+    p.dbg = Extents{};
+    p.dbg.q = (size_t)B * H * Nq * d;
+    p.dbg.kv = (size_t)B * H_kv * N * d;
+    p.dbg.lse = (size_t)B * H * Nq;
+    p.dbg.part = splits > 1 ? (size_t)splits * B * H * Nq * d : 0;
+    p.dbg.nseq = B;
 
     CUtensorMap tq, tk, tv;
     if (!make_bf16_map(&tq, q, d, G * Nq, B * H_kv, 128) ||
@@ -548,6 +558,20 @@ fa_status fa_fwd_decode(const void* q, const void* k_cache, const void* v_cache,
         return FA_ERR_CUDA;
     return FA_OK;
 }
+
+fa_status fa_selftest_bounds(int* buf, int n, int value, fa_stream_t stream) {
+    if (!kDebugChecks) return FA_ERR_UNSUPPORTED;  // checks compiled out: nothing to exercise
+    if (!buf || n < 1 || (reinterpret_cast<uintptr_t>(buf) & 3u)) return FA_ERR_INVALID_ARG;
+    fa_status st;
+    DeviceState* dev = current_device(&st);
+    if (!dev) return st;
+    if (fa::launch_bounds_selftest(buf, n, value, dev->err_flag,
+                                   reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return FA_ERR_CUDA;
+    return FA_OK;
+}
+
+int fa_debug_checks(void) { return kDebugChecks ? 1 : 0; }
 
 fa_status fa_selftest_wait_timeout(fa_stream_t stream) {
     fa_status st;

@@ -10,7 +10,8 @@
 //
 // Host code cannot use the array's name as a device address (on the host it only names a
 // stand-in object), so the device address is looked up once per device with
-// cudaGetSymbolAddress, with that device current, and handed to the kernels.
+// cudaGetSymbolAddress, with that device current, and handed to the kernels.  Under lazy
+// module loading that first lookup is also when the array is placed in device memory.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -47,9 +48,16 @@ fa_status scratch_for_current_device(void** out) {
             return FA_ERR_CUDA;
         s.supported = (major == 10 && minor == 0);
         if (s.supported) {
+            // With lazy module loading (the CUDA default since 12.2) this lookup is what loads
+            // this file's device image, and with it commits the scratch array: it can fail for
+            // lack of device memory, which is reported as FA_ERR_WORKSPACE.
             void* ptr = nullptr;
-            if (cudaGetSymbolAddress(&ptr, g_bwd_scratch) != cudaSuccess || ptr == nullptr)
-                return FA_ERR_CUDA;
+            const cudaError_t e = cudaGetSymbolAddress(&ptr, g_bwd_scratch);
+            if (e == cudaErrorMemoryAllocation) {
+                cudaGetLastError();  // not sticky: clear it so later calls start clean
+                return FA_ERR_WORKSPACE;
+            }
+            if (e != cudaSuccess || ptr == nullptr) return FA_ERR_CUDA;
             s.scratch = ptr;
         }
         s.ready = true;
@@ -121,6 +129,7 @@ extern "C" FA_API fa_status fa_bwd_noalloc(const void* q, const void* k, const v
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
     p.timeout_ns = fa::wait_timeout_ns();
+    p.dbg = fa::extents(B, H, H, N, d, 0, false);
 
     CUtensorMap tq, tk, tv, tdo;
     if (!fa::make_bf16_map(&tq, q, d, N, BH, 128) || !fa::make_bf16_map(&tk, k, d, N, BH, 128) ||

@@ -87,7 +87,7 @@ __global__ void __launch_bounds__(192, DecCfg<D>::CTAS_PER_SM)
     const int GNq = p.G * p.Nq;                      // query rows sharing this cache head
 
     int L = p.N;
-    if (p.cache_lens != nullptr) {
+    if (p.cache_lens != nullptr && in_bounds(p.err, b, 1, p.dbg.nseq)) {
         L = p.cache_lens[b];
         if (L < 1 || L > p.N) {
             if (threadIdx.x == 0 && split == 0 && blockIdx.y == 0) record_error(p.err, kErrInvalidArg);
@@ -361,6 +361,7 @@ __global__ void __launch_bounds__(192, DecCfg<D>::CTAS_PER_SM)
             const float inv_l = l > 0.f ? 1.0f / l : 0.f;
             const float lse_v = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
             if (p.splits == 1) {
+                const bool o_ok = valid && in_bounds(p.err, R * D, D, p.dbg.q);
                 __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + R * D;
 #pragma unroll 1
                 for (int q = 0; q < D / 32; ++q) {
@@ -370,7 +371,7 @@ __global__ void __launch_bounds__(192, DecCfg<D>::CTAS_PER_SM)
                         tmem_ld_wait();
                         reg_fence32(o);
                     }
-                    if (valid) {
+                    if (o_ok) {
                         uint32_t w[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i)
@@ -382,9 +383,10 @@ __global__ void __launch_bounds__(192, DecCfg<D>::CTAS_PER_SM)
                             dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
                     }
                 }
-                if (valid) p.lse[R] = lse_v;
+                if (valid && in_bounds(p.err, R, 1, p.dbg.lse)) p.lse[R] = lse_v;
             } else {
                 // partial of this split: O_s normalised by its own sum (0 if it saw no key)
+                const bool o_ok = valid && in_bounds(p.err, ((size_t)split * rows_total + R) * D, D, p.dbg.part);
                 float* orow = p.o_part + ((size_t)split * rows_total + R) * D;
 #pragma unroll 1
                 for (int q = 0; q < D / 32; ++q) {
@@ -397,7 +399,7 @@ __global__ void __launch_bounds__(192, DecCfg<D>::CTAS_PER_SM)
 #pragma unroll
                         for (int i = 0; i < 32; ++i) o[i] = 0u;
                     }
-                    if (valid) {
+                    if (o_ok) {
                         float4* dst = reinterpret_cast<float4*>(orow + q * 32);
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
@@ -407,7 +409,8 @@ __global__ void __launch_bounds__(192, DecCfg<D>::CTAS_PER_SM)
                                                  __uint_as_float(o[4 * i + 3]) * inv_l);
                     }
                 }
-                if (valid) p.lse_part[(size_t)split * rows_total + R] = lse_v;
+                if (valid && in_bounds(p.err, (size_t)split * rows_total + R, 1, p.dbg.part / D))
+                    p.lse_part[(size_t)split * rows_total + R] = lse_v;
             }
         } else {
             fail();
@@ -435,6 +438,10 @@ __global__ void __launch_bounds__(256) fa_decode_combine_kernel(const DecodePara
     const size_t rows_total = (size_t)p.B * p.H * p.Nq;
     const size_t R = (size_t)blockIdx.x * 8 + threadIdx.x / 32;
     if (R >= rows_total) return;
+    // every split's partial of this row, and the row of O and lse
+    if (!in_bounds(p.err, ((size_t)(p.splits - 1) * rows_total + R) * D, D, p.dbg.part) ||
+        !in_bounds(p.err, R * D, D, p.dbg.q) || !in_bounds(p.err, R, 1, p.dbg.lse))
+        return;
     float mx = -INFINITY;
     for (int s = lane; s < p.splits; s += 32) mx = fmaxf(mx, p.lse_part[s * rows_total + R]);
 #pragma unroll
@@ -476,14 +483,11 @@ cudaError_t launch_decode_d(const CUtensorMap& tq, const CUtensorMap& tk, const 
                             const DecodeParams& p, cudaStream_t stream, cudaEvent_t ev_start,
                             cudaEvent_t ev_stop) {
     using C = DecCfg<D>;
-    static bool configured = false;  // attribute set once per process (idempotent if raced)
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(fa_decode_kernel<D>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<uint64_t> configured{0};  // one bit per device
+    if (cudaError_t e = set_smem_limit_once(configured, C::SMEM_BYTES,
+                                            fa_decode_kernel<D>);
+        e != cudaSuccess)
+        return e;
     const dim3 grid(p.splits, p.H_kv * p.n_mtiles, p.B);  // splits in units of C::BN blocks
     if (ev_start) cudaEventRecord(ev_start, stream);
     fa_decode_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);

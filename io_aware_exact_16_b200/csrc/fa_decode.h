@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "fa_internal.h"
+
 namespace fa {
 
 struct DecodeParams {
@@ -23,6 +25,7 @@ struct DecodeParams {
     float scale_log2;       // scale * log2(e)
     int causal;
     uint64_t timeout_ns;
+    Extents dbg;            // buffer sizes for the FA_DEBUG index checks
 };
 
 // Query tile map: q [B, H, Nq, d] seen as (d, G*Nq, B*H_kv); cache maps as make_bf16_map.

@@ -347,9 +347,9 @@ __global__ void __launch_bounds__(192, 1)
         if (__all_sync(0xffffffffu, ok)) {
             tc_fence_after();
             const float inv_l = l > 0.f ? 1.0f / l : 0.f;
-            const bool in_range = row < ext.Lq;
-            __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) +
-                                  row_of(packed, b, h, p.H, p.N, ext.t0, in_range ? row : 0) * D;
+            const size_t o_off = row_of(packed, b, h, p.H, p.N, ext.t0, row < ext.Lq ? row : 0) * D;
+            const bool in_range = row < ext.Lq && in_bounds(p.err, o_off, D, p.dbg.q);
+            __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + o_off;
 #pragma unroll 1
             for (int q = 0; q < D / 32; ++q) {
                 uint32_t o[32];
@@ -368,10 +368,10 @@ __global__ void __launch_bounds__(192, 1)
                         dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
                 }
             }
-            if (in_range) {
+            const size_t l_off = lse_of(packed, b, h, p.H, p.N, p.T, ext.t0, row);
+            if (in_range && in_bounds(p.err, l_off, 1, p.dbg.lse)) {
                 // lse in natural-log units: (m + log2 l) * ln 2
-                p.lse[lse_of(packed, b, h, p.H, p.N, p.T, ext.t0, row)] =
-                    l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+                p.lse[l_off] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
             }
         } else {
             fail();
@@ -391,14 +391,11 @@ template <bool PACKED>
 cudaError_t launch_d256(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                         const FwdParams& p, int B, cudaStream_t stream) {
     using C = Fwd256Cfg;
-    static bool configured = false;  // attribute set once per process (idempotent if raced)
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(fa_fwd_d256_kernel<PACKED>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<uint64_t> configured{0};  // one bit per device
+    if (cudaError_t e = set_smem_limit_once(configured, C::SMEM_BYTES,
+                                            fa_fwd_d256_kernel<PACKED>);
+        e != cudaSuccess)
+        return e;
     dim3 grid((p.N + C::BM - 1) / C::BM, p.H, B);
     fa_fwd_d256_kernel<PACKED><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
     return cudaGetLastError();

@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(384, 1)
     const int q_base = cta_x * C::ROWS_PER_CTA;
 
     int L = p.N;
-    if (p.seqlens != nullptr) {
+    if (p.seqlens != nullptr && in_bounds(p.err, b, 1, p.dbg.nseq)) {
         L = p.seqlens[b];
         if (L < 1 || L > p.N) {
             if (threadIdx.x == 0 && h == 0 && cta_x == 0) record_error(p.err, kErrInvalidArg);
@@ -309,8 +309,9 @@ __global__ void __launch_bounds__(384, 1)
         const int nt = t ? nblk1 : nblk0;
         const int row = q_base + t * C::BM + r;
         const int lim = p.causal ? min(L, row + 1) : L;
-        const float qd = p.q_descale ? p.q_descale[bh] : 1.0f;
-        const float kd = p.k_descale ? p.k_descale[bh_kv] : 1.0f;
+        const float qd = p.q_descale && in_bounds(p.err, bh, 1, p.dbg.heads_q) ? p.q_descale[bh] : 1.0f;
+        const float kd = p.k_descale && in_bounds(p.err, bh_kv, 1, p.dbg.heads_kv)
+                             ? p.k_descale[bh_kv] : 1.0f;
         const float c = p.scale_log2 * qd * kd;  // scores of the codes -> log2 units
         float m = -INFINITY;  // running max of S * c, possibly stale by <= THRESH
         float l = 0.f;        // running sum of p' = exp2(S * c - m + P_OFFSET)
@@ -410,11 +411,12 @@ __global__ void __launch_bounds__(384, 1)
         if (ok) ok = mbar_wait(&bar_ofull[t], (nt - 1) & 1, p.timeout_ns, abort_flag);
         if (__all_sync(0xffffffffu, ok)) {
             tc_fence_after();
-            const float vd = p.v_descale ? p.v_descale[bh_kv] : 1.0f;
+            const float vd = p.v_descale && in_bounds(p.err, bh_kv, 1, p.dbg.heads_kv)
+                                 ? p.v_descale[bh_kv] : 1.0f;
             const float mul = l > 0.f ? vd / l : 0.f;
-            const bool in_range = row < p.N;
-            __nv_bfloat16* orow =
-                reinterpret_cast<__nv_bfloat16*>(p.o) + ((size_t)bh * p.N + (in_range ? row : 0)) * D;
+            const size_t o_off = ((size_t)bh * p.N + (row < p.N ? row : 0)) * D;
+            const bool in_range = row < p.N && in_bounds(p.err, o_off, D, p.dbg.q);
+            __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + o_off;
 #pragma unroll
             for (int q = 0; q < D / 32; ++q) {
                 uint32_t o[32];
@@ -433,7 +435,7 @@ __global__ void __launch_bounds__(384, 1)
                         dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
                 }
             }
-            if (in_range) {
+            if (in_range && in_bounds(p.err, (size_t)bh * p.N + row, 1, p.dbg.lse)) {
                 // l' carries the 2^P_OFFSET of p': lse = (m + log2 l' - P_OFFSET) * ln 2
                 p.lse[(size_t)bh * p.N + row] =
                     l > 0.f ? (m + __log2f(l) - C::P_OFFSET) * 0.69314718055994531f : -INFINITY;
@@ -457,14 +459,11 @@ __global__ void __launch_bounds__(384, 1)
 cudaError_t launch_fwd_fp8(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                            const Fp8Params& p, int B, cudaStream_t stream) {
     using C = Fp8Cfg;
-    static bool configured = false;  // attribute set once per process (idempotent if raced)
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(fa_fwd_fp8_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<uint64_t> configured{0};  // one bit per device
+    if (cudaError_t e = set_smem_limit_once(configured, C::SMEM_BYTES,
+                                            fa_fwd_fp8_kernel);
+        e != cudaSuccess)
+        return e;
     dim3 grid((p.N + C::ROWS_PER_CTA - 1) / C::ROWS_PER_CTA, p.H, B);
     fa_fwd_fp8_kernel<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
     return cudaGetLastError();

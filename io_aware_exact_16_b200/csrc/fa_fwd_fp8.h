@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "fa_internal.h"
+
 namespace fa {
 
 struct Fp8Params {
@@ -20,6 +22,7 @@ struct Fp8Params {
     float scale_log2;        // scale * log2(e)
     int causal;
     uint64_t timeout_ns;
+    Extents dbg;            // buffer sizes for the FA_DEBUG index checks
 };
 
 // Tensor maps: e4m3 [B*Hx, N, 128] as bytes, box 128 x 128 rows, 128-byte swizzle.

@@ -173,3 +173,17 @@ def test_wait_selftest_reports_a_missing_device_instead_of_launching():
         pytest.skip("a device is present; the GPU test covers the launch")
     st = fa.raw_library().fa_selftest_wait_timeout(None)
     assert st in (fa.FA_ERR_CUDA, fa.FA_ERR_UNSUPPORTED)
+
+
+def test_debug_build_exports_the_same_symbols_and_reports_its_checks():
+    """libfa_debug.so (FA_DEBUG: index checks on every plain global access) is the same C ABI;
+    fa_debug_checks tells the two builds apart, and the release build refuses the bounds
+    self-test (its checks are compiled out) before touching a device."""
+    dbg = fa.debug_library()
+    for name in declared_symbols():
+        assert hasattr(dbg, name), name
+    assert dbg.fa_debug_checks() == 1
+    assert fa.raw_library().fa_debug_checks() == 0
+    assert fa.raw_library().fa_selftest_bounds(16, 8, 1, None) == fa.FA_ERR_UNSUPPORTED
+    assert dbg.fa_selftest_bounds(None, 8, 1, None) == fa.FA_ERR_INVALID_ARG
+    assert dbg.fa_selftest_bounds(16, 0, 1, None) == fa.FA_ERR_INVALID_ARG
