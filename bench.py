@@ -50,6 +50,13 @@ WORKLOADS = {
     "gqa-N4096-H32-kv8-d128": lambda: workloads.Workload(
         "gqa non-causal B2 H32 Hkv8 N4096 d128", 2, 32, 4096, 128, False, 1040, H_kv=8),
 }
+for _N in workloads.SWEEP_N:
+    for _H, _d in workloads.SWEEP_HD:
+        for _c in (False, True):
+            WORKLOADS.setdefault(f"sweep-N{_N}-H{_H}-d{_d}" + ("-causal" if _c else ""),
+                                 (lambda N=_N, H=_H, d=_d, c=_c: workloads.sweep(N, H, d, c)))
+SWEEP_NAMES = [f"sweep-N{N}-H{H}-d{d}" + ("-causal" if c else "")
+               for N in workloads.SWEEP_N for (H, d) in workloads.SWEEP_HD for c in (False, True)]
 DEFAULT_WORKLOAD = "sweep-N4096-H16-d128"
 
 
@@ -63,6 +70,39 @@ def flops_per_step(w: workloads.Workload, seqlens=None) -> tuple[float, float]:
     if w.causal:
         fwd /= 2.0
     return fwd, 2.5 * fwd
+
+
+def tensor_peak(peaks: dict, src: str, timed_s: float, clocks: dict | None) -> tuple[float, str]:
+    """The bf16 tensor peak a kernel timed in this run is set against.  The measured burst
+    figure (a GEMM timed alone) applies to a timed region shorter than a second whose clock
+    record shows no power capping; a longer or power-capped region is set against the
+    sustained figure (a seconds-long GEMM loop under the power cap)."""
+    reasons = (clocks or {}).get("reasons", [])
+    if timed_s < 1.0 and "sw_power_cap" not in reasons:
+        return float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])), f"{src} bf16 burst"
+    return (float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])),
+            f"{src} bf16 sustained")
+
+
+def roofline_tensor(kernel: str, achieved: float, kernel_ms: float, peaks: dict, src: str,
+                    timed_s: float, clocks: dict | None, traffic, scale: float = 1.0) -> dict:
+    """Roofline object of a tensor-bound kernel: `frac` against the peak that applies (see
+    tensor_peak), plus both measured fractions and the share of the nominal dense peak.
+    `scale` multiplies the bf16 peaks (2 for e4m3, the nominal ratio)."""
+    peak, which = tensor_peak(peaks, src, timed_s, clocks)
+    burst = scale * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    sust = scale * float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    peak *= scale
+    source = which + (" (MEASURED_PEAKS.json)" if src == "measured" else " (no MEASURED_PEAKS.json)")
+    if scale != 1.0:
+        source += f" x {scale:g} (nominal e4m3 / bf16 ratio)"
+    return {"kernel": kernel, "bound": "tensor", "achieved": round(achieved, 2),
+            "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+            "peak_source": source,
+            "frac_of_burst": round(achieved / burst, 4),
+            "frac_of_sustained": round(achieved / sust, 4),
+            "pct_of_2250": round(100.0 * achieved / (scale * NOMINAL_PEAK_TFLOPS), 2),
+            "kernel_ms": round(kernel_ms, 4), "traffic": traffic}
 
 
 def load_peaks() -> tuple[dict, str]:
@@ -274,61 +314,68 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     # memory and its results (O, dQ, dK, dV) out to pinned host memory.  The copies run on their
     # own streams over two device buffer sets, so step s+1's inputs travel while step s
     # computes and step s-1's results travel back, as a training input pipeline would do.
-    def device_set():
-        return {"q": torch.empty_like(q), "k": torch.empty_like(k), "v": torch.empty_like(v),
-                "do": torch.empty_like(do), "o": torch.empty_like(o),
-                "lse": torch.empty_like(lse), "dq": torch.empty_like(dq),
-                "dk": torch.empty_like(dk), "dv": torch.empty_like(dv),
-                "ws": torch.empty_like(ws)}
+    def e2e_leg():
+        def device_set():
+            return {"q": torch.empty_like(q), "k": torch.empty_like(k), "v": torch.empty_like(v),
+                    "do": torch.empty_like(do), "o": torch.empty_like(o),
+                    "lse": torch.empty_like(lse), "dq": torch.empty_like(dq),
+                    "dk": torch.empty_like(dk), "dv": torch.empty_like(dv),
+                    "ws": torch.empty_like(ws)}
 
-    sets = [device_set(), device_set()]
-    outs = ("o", "dq", "dk", "dv")
-    host_out = [{n: torch.empty(sets[0][n].shape, dtype=sets[0][n].dtype).pin_memory()
-                 for n in outs} for _ in range(2)]
-    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
-    d2h = sum(host_out[0][n].numel() * host_out[0][n].element_size() for n in outs)
-    e2e_steps = max(1, min(args.steps, 10))
-    copy_in = torch.cuda.Stream(dev)
-    copy_out = torch.cuda.Stream(dev)
-    ev = lambda: torch.cuda.Event()  # noqa: E731
-    in_done = [ev() for _ in range(e2e_steps)]
-    comp_done = [ev() for _ in range(e2e_steps)]
-    out_done = [ev() for _ in range(e2e_steps)]
-    barrier()
-    torch.cuda.synchronize(dev)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    copy_in.wait_event(e0)
-    for s_ in range(e2e_steps):
-        bset = sets[s_ % 2]
-        with torch.cuda.stream(copy_in):
+        sets = [device_set(), device_set()]
+        outs = ("o", "dq", "dk", "dv")
+        host_out = [{n: torch.empty(sets[0][n].shape, dtype=sets[0][n].dtype).pin_memory()
+                     for n in outs} for _ in range(2)]
+        h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+        d2h = sum(host_out[0][n].numel() * host_out[0][n].element_size() for n in outs)
+        e2e_steps = max(1, min(args.steps, 10))
+        copy_in = torch.cuda.Stream(dev)
+        copy_out = torch.cuda.Stream(dev)
+        ev = lambda: torch.cuda.Event()  # noqa: E731
+        in_done = [ev() for _ in range(e2e_steps)]
+        comp_done = [ev() for _ in range(e2e_steps)]
+        out_done = [ev() for _ in range(e2e_steps)]
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        copy_in.wait_event(e0)
+        for s_ in range(e2e_steps):
+            bset = sets[s_ % 2]
+            with torch.cuda.stream(copy_in):
+                if s_ >= 2:
+                    copy_in.wait_event(comp_done[s_ - 2])  # step s-2 has read this set's inputs
+                for n in ("q", "k", "v", "do"):
+                    bset[n].copy_(pinned[n], non_blocking=True)
+                in_done[s_].record(copy_in)
+            stream.wait_event(in_done[s_])
             if s_ >= 2:
-                copy_in.wait_event(comp_done[s_ - 2])  # step s-2 has read this set's inputs
-            for n in ("q", "k", "v", "do"):
-                bset[n].copy_(pinned[n], non_blocking=True)
-            in_done[s_].record(copy_in)
-        stream.wait_event(in_done[s_])
-        if s_ >= 2:
-            stream.wait_event(out_done[s_ - 2])  # step s-2's results have left this set
-        fa.forward(bset["q"], bset["k"], bset["v"], causal=w.causal, seqlens=sl, scale=w.scale,
-                   out=bset["o"], lse=bset["lse"])
-        fa.backward(bset["q"], bset["k"], bset["v"], bset["o"], bset["do"], bset["lse"],
-                    causal=w.causal, seqlens=sl, scale=w.scale, dq=bset["dq"], dk=bset["dk"],
-                    dv=bset["dv"], workspace=bset["ws"])
-        comp_done[s_].record(stream)
-        with torch.cuda.stream(copy_out):
-            copy_out.wait_event(comp_done[s_])
-            for n in outs:
-                host_out[s_ % 2][n].copy_(bset[n], non_blocking=True)
-            out_done[s_].record(copy_out)
-    stream.wait_event(out_done[e2e_steps - 1])
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    e2e_ms = e0.elapsed_time(e1)
-    if fa.check_device_error(dev) != 0:
-        raise RuntimeError("device error flag set in the end-to-end leg")
+                stream.wait_event(out_done[s_ - 2])  # step s-2's results have left this set
+            fa.forward(bset["q"], bset["k"], bset["v"], causal=w.causal, seqlens=sl, scale=w.scale,
+                       out=bset["o"], lse=bset["lse"])
+            fa.backward(bset["q"], bset["k"], bset["v"], bset["o"], bset["do"], bset["lse"],
+                        causal=w.causal, seqlens=sl, scale=w.scale, dq=bset["dq"], dk=bset["dk"],
+                        dv=bset["dv"], workspace=bset["ws"])
+            comp_done[s_].record(stream)
+            with torch.cuda.stream(copy_out):
+                copy_out.wait_event(comp_done[s_])
+                for n in outs:
+                    host_out[s_ % 2][n].copy_(bset[n], non_blocking=True)
+                out_done[s_].record(copy_out)
+        stream.wait_event(out_done[e2e_steps - 1])
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e2e_ms = e0.elapsed_time(e1)
+        if fa.check_device_error(dev) != 0:
+            raise RuntimeError("device error flag set in the end-to-end leg")
+        return e2e_ms, h2d, d2h, e2e_steps
+
+    if args.skip_e2e:
+        e2e_ms, h2d, d2h, e2e_steps = 0.0, 0, 0, 0
+    else:
+        e2e_ms, h2d, d2h, e2e_steps = e2e_leg()
 
     elapsed_ms, e2e_ms, fwd_ms, bwd_ms, fwd_kernel_ms, bwd_kernel_ms = reduce_max(
         [elapsed_ms, e2e_ms, fwd_ms, bwd_ms, fwd_kernel_ms, bwd_kernel_ms], world, dev)
@@ -336,7 +383,6 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
         return None
 
     peaks, peak_src = load_peaks()
-    sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     value = step_flops * args.steps * world / (elapsed_ms * 1e-3) / 1e12
     ms_per_step = elapsed_ms / args.steps
     bwd_tflops = bwd_flops / (bwd_ms * 1e-3) / 1e12
@@ -344,6 +390,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     # every backward GEMM (recompute S, dP, dV, dK, dQ) runs in the fused kernel
     bwd_kernel_tflops = bwd_flops / (bwd_kernel_ms * 1e-3) / 1e12
     fwd_kernel_tflops = fwd_flops / (fwd_kernel_ms * 1e-3) / 1e12
+    clock_summary = clocks.summary()
+    timed_s = elapsed_ms * 1e-3
     wname = args.workload
     traffic = dram_traffic("fa_bwd_kernel", wname)
     line = {
@@ -371,28 +419,21 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
                    "fwd_pct_of_2250": round(100 * fwd_tflops / NOMINAL_PEAK_TFLOPS, 2),
                    "bwd_pct_of_2250": round(100 * bwd_tflops / NOMINAL_PEAK_TFLOPS, 2),
                    "step_ms_p10_p50_p90": [round(_pct(step_ms, q), 4) for q in (10, 50, 90)]},
-        "roofline": {
-            "kernel": "fa_bwd_kernel (fused backward: all five backward GEMMs)",
-            "bound": "tensor", "achieved": round(bwd_kernel_tflops, 2),
-            "peak": sustained, "unit": "TFLOP/s",
-            "frac": round(bwd_kernel_tflops / sustained, 4),
-            "peak_source": f"{peak_src} bf16 sustained (MEASURED_PEAKS.json)",
-            "kernel_ms": round(bwd_kernel_ms, 4),
-            "traffic": traffic,
-        },
-        "roofline_fwd": {
-            "kernel": "fa_fwd_kernel", "bound": "tensor", "achieved": round(fwd_kernel_tflops, 2),
-            "peak": sustained, "unit": "TFLOP/s", "frac": round(fwd_kernel_tflops / sustained, 4),
-            "kernel_ms": round(fwd_kernel_ms, 4),
-            "traffic": dram_traffic("fa_fwd_kernel", wname),
-        },
-        "e2e": {"value": round(step_flops * e2e_steps * world / (e2e_ms * 1e-3) / 1e12, 2),
+        "roofline": roofline_tensor("fa_bwd_kernel (fused backward: all five backward GEMMs)",
+                                    bwd_kernel_tflops, bwd_kernel_ms, peaks, peak_src, timed_s,
+                                    clock_summary, traffic),
+        "roofline_fwd": roofline_tensor("fa_fwd_kernel", fwd_kernel_tflops, fwd_kernel_ms, peaks,
+                                        peak_src, timed_s, clock_summary,
+                                        dram_traffic("fa_fwd_kernel", wname)),
+        "e2e": {"value": round(step_flops * e2e_steps * world / (max(e2e_ms, 1e-9) * 1e-3) / 1e12, 2),
                 "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps, "copies": "pinned host memory, own streams, overlapped "
                                               "with the neighbouring steps' compute"},
         "gpu_launches": 4 * args.steps,
-        "clocks": clocks.summary(),
+        "clocks": clock_summary,
     }
+    if args.skip_e2e:
+        del line["e2e"]
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_heads)
     return line
@@ -490,6 +531,7 @@ class Row:
     launches: int                # our kernels per step
     cpu: Callable[[], dict]      # the oracle on a bounded sample: {"amount", "seconds", "sample"}
     traffic_key: str | None = None
+    peak_scale: float = 1.0      # tensor rows: multiple of the bf16 peaks (2 for e4m3)
 
 
 def _pinned_pair(t: torch.Tensor):
@@ -605,7 +647,8 @@ def row_fwd_fp8(rank: int, dev) -> Row:
                step=lambda mark: (mark(), fa.forward_fp8(q, k, v, qd, kd, vd, scale=w.scale,
                                                          out=o, lse=lse)),
                h2d=[(q, f.q.pin_memory()), (k, f.k.pin_memory()), (v, f.v.pin_memory())],
-               d2h=[_pinned_pair(o)], launches=1, cpu=cpu, traffic_key="fa_fwd_fp8_kernel")
+               d2h=[_pinned_pair(o)], launches=1, cpu=cpu, traffic_key="fa_fwd_fp8_kernel",
+               peak_scale=2.0)
 
 
 def row_decode(rank: int, dev) -> Row:
@@ -751,6 +794,7 @@ def run_row(args, rank: int, world: int, local_rank: int) -> dict | None:
         return None
 
     scale_unit = 1e12 if row.unit == "TFLOP/s" else 1e9
+    clock_summary = clocks.summary()
     value = row.amount * args.steps * world / (elapsed_ms * 1e-3) / scale_unit
     achieved = row.kernel_amount / (kernel_ms * 1e-3) / scale_unit
     traffic = dram_traffic(row.traffic_key, row.config["workload"]) if row.traffic_key else None
@@ -761,17 +805,20 @@ def run_row(args, rank: int, world: int, local_rank: int) -> dict | None:
         "scaling": "weak", "vs_baseline": None, "dtype": row.dtype,
         "data": "synthetic (seeded N(0,1) draws)", "row": args.row,
         "config": dict(row.config, parallelism=f"independent batches x{world}"),
-        "roofline": {"kernel": row.kernel, "bound": row.bound, "achieved": round(achieved, 2),
-                     "peak": row.peak, "unit": row.unit, "frac": round(achieved / row.peak, 4),
-                     "peak_source": row.peak_source, "kernel_ms": round(kernel_ms, 4),
-                     "traffic": traffic},
+        "roofline": ({"kernel": row.kernel, "bound": row.bound, "achieved": round(achieved, 2),
+                      "peak": row.peak, "unit": row.unit, "frac": round(achieved / row.peak, 4),
+                      "peak_source": row.peak_source, "kernel_ms": round(kernel_ms, 4),
+                      "traffic": traffic} if row.bound != "tensor" else
+                     roofline_tensor(row.kernel, achieved, kernel_ms, *load_peaks(),
+                                     elapsed_ms * 1e-3, clock_summary, traffic,
+                                     scale=row.peak_scale)),
         "e2e": {"value": round(row.amount * e2e_steps * world / (e2e_ms * 1e-3) / scale_unit, 2),
                 "unit": row.unit,
                 "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t, _ in row.h2d),
                 "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t, _ in row.d2h),
                 "steps": e2e_steps},
         "gpu_launches": row.launches * args.steps,
-        "clocks": clocks.summary(),
+        "clocks": clock_summary,
     }
     if not args.no_cpu_baseline:
         import oracle
@@ -815,7 +862,32 @@ def run_row_reference(args, rank: int, world: int) -> dict | None:
     }
 
 
-def main() -> int:
+def relaunch(n: int, argv: list[str], timeout_s: int) -> int:
+    """`--gpus N` without a launcher: start N ranks of this script with torch.distributed.run
+    (one process per GPU, rendezvous on 127.0.0.1) and pass rank 0's JSON line through.  Every
+    rank's timing is reduced to the maximum over ranks inside the job."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = ["timeout", "-k", "60", str(timeout_s), sys.executable, "-m", "torch.distributed.run",
+           "--nnodes=1", f"--nproc-per-node={n}", "--master-addr=127.0.0.1",
+           f"--master-port={port}", os.path.abspath(__file__)] + argv
+    return subprocess.call(cmd)
+
+
+def run_selftest_ranks(args, rank: int, world: int) -> dict | None:
+    """Host-side check of the multi-rank path without a GPU (gloo): each rank reports a
+    different fake time; rank 0 returns the line the real run would print, with the maximum."""
+    fake_ms = [10.0 + rank, 100.0 - rank]
+    elapsed_ms, other = reduce_max(fake_ms, world)
+    if rank != 0:
+        return None
+    return {"metric": METRIC, "selftest": True, "n_gpus": world, "scaling": "weak",
+            "ms_max_over_ranks": [elapsed_ms, other]}
+
+
+def main(argv: list[str] | None = None) -> int:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
@@ -826,33 +898,61 @@ def main() -> int:
     ap.add_argument("--row", choices=["train"] + sorted(ROWS), default="train",
                     help="train: forward + backward step (default); others: the further "
                          "entry points, each on its own workload")
+    ap.add_argument("--sweep", action="store_true",
+                    help="one training line per throughput-sweep point (N 512..16384 x "
+                         "(H16, d128), (H32, d64) x causal and not), without the end-to-end "
+                         "leg and the oracle")
     ap.add_argument("--cpu-heads", type=int, default=12)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    args = ap.parse_args()
-    if args.warmup < 3 and args.impl == "ours":
+    ap.add_argument("--skip-e2e", action="store_true", help=argparse.SUPPRESS)
+    ap.add_argument("--selftest-ranks", action="store_true",
+                    help="check the multi-rank launch and max-over-ranks logic on CPU (gloo)")
+    ap.add_argument("--launch-timeout", type=int, default=1800,
+                    help="seconds before a self-launched multi-rank job is stopped")
+    raw = sys.argv[1:] if argv is None else argv
+    args = ap.parse_args(raw)
+    if args.warmup < 3 and args.impl == "ours" and not args.selftest_ranks:
         ap.error("--warmup must be >= 3")
 
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        return relaunch(args.gpus, raw, args.launch_timeout)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if world != args.gpus:
-        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
-    distributed = world > 1 and args.impl == "ours"
+        print(f"error: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+        return 2
+    distributed = world > 1 and (args.impl == "ours" or args.selftest_ranks)
     if distributed:
         import datetime
         os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
-        torch.cuda.set_device(local_rank)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    try:
-        if args.row != "train":
-            line = (run_row_reference(args, rank, world) if args.impl == "reference"
-                    else run_row(args, rank, world, local_rank))
-        elif args.impl == "reference":
-            line = run_reference(args, rank, world)
+        if args.selftest_ranks:
+            torch.distributed.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
         else:
-            line = run_ours(args, rank, world, local_rank)
-        if line is not None:
-            print(json.dumps(line), flush=True)
+            torch.cuda.set_device(local_rank)
+            torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        if args.selftest_ranks:
+            lines = [run_selftest_ranks(args, rank, world)]
+        elif args.row != "train":
+            lines = [run_row_reference(args, rank, world) if args.impl == "reference"
+                     else run_row(args, rank, world, local_rank)]
+        elif args.impl == "reference":
+            lines = [run_reference(args, rank, world)]
+        elif args.sweep:
+            lines = []
+            for name in SWEEP_NAMES:
+                pa = argparse.Namespace(**vars(args))
+                pa.workload, pa.skip_e2e, pa.no_cpu_baseline = name, True, True
+                line = run_ours(pa, rank, world, local_rank)
+                if line is not None:
+                    line["row"] = "sweep"
+                    print(json.dumps(line), flush=True)
+        else:
+            lines = [run_ours(args, rank, world, local_rank)]
+        for line in lines:
+            if line is not None:
+                print(json.dumps(line), flush=True)
     finally:
         if distributed:
             torch.distributed.destroy_process_group()

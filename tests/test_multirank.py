@@ -49,3 +49,24 @@ def test_two_ranks_take_independent_batches_and_max_time():
         (s0, *shape0, f0), (s1, *shape1, f1) = gathered
         assert shape0 == shape1          # same per-GPU shape: weak scaling
         assert s0 != s1 and f0 != f1     # different seeded data per rank
+
+
+def test_bench_launches_its_own_ranks():
+    """`bench.py --gpus 2` without a launcher starts two ranks itself (torch.distributed.run on
+    127.0.0.1); the rank self-test runs the same launch and max-over-ranks path on gloo, and
+    rank 0 alone prints one line that reports both ranks."""
+    import json
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2",
+                          "--selftest-ranks", "--launch-timeout", "240"],
+                         capture_output=True, text=True, timeout=300, env=env, cwd=root)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, out.stdout
+    line = json.loads(lines[0])
+    assert line["n_gpus"] == 2
+    assert line["ms_max_over_ranks"] == [11.0, 100.0]  # rank 1's first, rank 0's second value
