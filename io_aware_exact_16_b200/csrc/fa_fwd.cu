@@ -31,11 +31,6 @@
 #include "fa_internal.h"
 #include "sm100.cuh"
 
-// Of every 4 pairs of scores, this many take their exponential on the FMA pipe (exp2_fma2)
-// and the rest on the MUFU unit, so the two units share the softmax's exponentials.
-#ifndef FA_FWD_EXP2_FMA_OF_4
-#define FA_FWD_EXP2_FMA_OF_4 0
-#endif
 // The softmax releases each block's P to the MMA thread in this many parts of BN / parts keys,
 // so that the P V MMAs of the first parts run while it computes the later ones.
 #ifndef FA_FWD_P_PARTS
@@ -64,11 +59,20 @@ struct FwdCfg {
     static constexpr int SMEM_BAR = SMEM_V + STAGES * KV_TILE_BYTES;
     static constexpr int P_PARTS = FA_FWD_P_PARTS;  // P released in parts of BN / P_PARTS keys
     static_assert(P_PARTS == 2 || P_PARTS == 4, "P is released in halves or quarters");
-    static constexpr int NUM_BARS = 1 + 4 * STAGES + 2 + 2 + 2 + 2 * (P_PARTS - 1) + 1;
+    // q, k/v full and empty per stage, s/p/o full per tile, P parts, done, and the persistent
+    // kernel's Q-empty barrier
+    static constexpr int NUM_BARS = 1 + 4 * STAGES + 2 + 2 + 2 + 2 * (P_PARTS - 1) + 1 + 1;
     static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;  // + alignment slack
     static constexpr int THREADS = 384;
     static constexpr uint32_t REGS_SOFTMAX = 224, REGS_OTHER = 56;
+    // The persistent kernel's MMA and TMA threads carry loop state across units and spill at
+    // 56 registers; there the split is 2 x 208 + 88 (the same 3 x 168 launched).
+#ifndef FA_FWD_PERSIST_REGS_SOFTMAX
+#define FA_FWD_PERSIST_REGS_SOFTMAX 208
+#endif
+    static constexpr uint32_t REGS_SOFTMAX_PERSIST = FA_FWD_PERSIST_REGS_SOFTMAX;
+    static constexpr uint32_t REGS_OTHER_PERSIST = 504 - 2 * REGS_SOFTMAX_PERSIST;
     static constexpr uint32_t TMEM_COLS = 512;
     // tensor-memory column of S_t / O_t for query tile t
     __device__ static constexpr uint32_t tm_s(int t) { return t ? 128u : 0u; }
@@ -113,6 +117,14 @@ __device__ __forceinline__ CtaCoords cta_coords(bool grouped) {
         c.b = (int)bz;
     }
     return c;
+}
+
+// An opaque copy of v: values derived from it are recomputed where they are used instead of
+// being kept live across the loop in between.
+__device__ __forceinline__ int opaque(int v) {
+    int r;
+    asm volatile("mov.b32 %0, %1;" : "=r"(r) : "r"(v));
+    return r;
 }
 
 template <int D, bool PACKED, bool GROUPED>
@@ -429,9 +441,7 @@ __global__ void __launch_bounds__(384, 1)
                     const int e0 = part * 2 * WP + 2 * i;
                     const float2 x = ffma2(make_float2(__uint_as_float(s[e0]),
                                                        __uint_as_float(s[e0 + 1])), c2, nm2);
-                    const float2 e = (i % 4 < FA_FWD_EXP2_FMA_OF_4)
-                                         ? exp2_fma2(x)
-                                         : make_float2(ex2(x.x), ex2(x.y));
+                    const float2 e = make_float2(ex2(x.x), ex2(x.y));
                     acc[i % 4] = fadd2(acc[i % 4], e);
                     pk[i] = pack_bf16x2(e.x, e.y);
                 }
@@ -492,17 +502,383 @@ __global__ void __launch_bounds__(384, 1)
     }
 }
 
+// Persistent forward for launches whose work units all cost the same: head-major, no causal
+// mask, no per-sequence key lengths (every tile pair sees all N keys).  One CTA per SM walks
+// the units blockIdx.x, blockIdx.x + gridDim.x, ... (tile pair x of head bh, head by head, so
+// a few heads' K and V stay in L2).  Per key block the arithmetic is fa_fwd_kernel's; across
+// units the K/V ring and every barrier phase carry over, the Q tiles are reloaded as soon as the
+// previous unit's last score MMA has completed (bar_qempty), and a unit's epilogue overlaps the
+// next unit's Q load and first score MMAs.  A unit's first P V of tile t overwrites O_t only
+// after the softmax threads of tile t have read O_t in their epilogue: they release P_t(0) of
+// the next unit after that.
+template <int D>
+__global__ void __launch_bounds__(384, 1)
+    fa_fwd_persist_kernel(const __grid_constant__ CUtensorMap tmQ,
+                          const __grid_constant__ CUtensorMap tmK,
+                          const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+    using C = FwdCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    const int nx = (p.N + C::ROWS_PER_CTA - 1) / C::ROWS_PER_CTA;  // tile pairs per head
+    const int n_units = nx * p.B * p.H;
+    const int nblk = (p.N + C::BN - 1) / C::BN;  // key blocks of every query tile
+
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_BAR);
+    uint64_t* bar_q = bars;
+    uint64_t* bar_kfull = bars + 1;
+    uint64_t* bar_kempty = bar_kfull + C::STAGES;
+    uint64_t* bar_vfull = bar_kempty + C::STAGES;
+    uint64_t* bar_vempty = bar_vfull + C::STAGES;
+    uint64_t* bar_sfull = bar_vempty + C::STAGES;  // [2]
+    uint64_t* bar_pfull = bar_sfull + 2;            // [2]
+    uint64_t* bar_ofull = bar_pfull + 2;            // [2]
+    uint64_t* bar_ppart = bar_ofull + 2;            // [2][P_PARTS-1]
+    uint64_t* bar_done = bar_ppart + 2 * (C::P_PARTS - 1);
+    uint64_t* bar_qempty = bar_done + 1;  // the unit's score MMAs are done: Q may be reloaded
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SMEM_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::SMEM_MISC + 4);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_q, 1);
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&bar_kfull[s], 1);
+            mbar_init(&bar_kempty[s], 1);
+            mbar_init(&bar_vfull[s], 1);
+            mbar_init(&bar_vempty[s], 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&bar_sfull[t], 1);
+            mbar_init(&bar_pfull[t], C::BM);
+            mbar_init(&bar_ofull[t], 1);
+            for (int q = 0; q + 1 < C::P_PARTS; ++q) mbar_init(&bar_ppart[t * (C::P_PARTS - 1) + q], C::BM);
+        }
+        mbar_init(bar_done, 1);
+        mbar_init(bar_qempty, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 8) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    auto fail = [&]() {
+        record_error(p.err, kErrTimeout);
+        *abort_flag = 1;
+    };
+
+    if (warp >= 8) {
+      regs_decrease<C::REGS_OTHER_PERSIST>();
+      if (warp == 9) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_tensormap(&tmQ);
+            prefetch_tensormap(&tmK);
+            prefetch_tensormap(&tmV);
+            int g = 0;   // K/V blocks whose V copy was issued (position in the ring)
+            int gk = 0;  // K copies issued
+            int uc = 0;  // units started
+            bool ok = true;
+            for (int lin = blockIdx.x; ok && lin < n_units; lin += gridDim.x, ++uc) {
+                const int bh = lin / nx;
+                const int q_base = (lin - bh * nx) * C::ROWS_PER_CTA;
+                const int bkv = (bh / p.H) * p.H_kv + (bh % p.H) / (p.H / p.H_kv);
+                if (uc > 0 && !(ok = mbar_wait(bar_qempty, (uc - 1) & 1, p.timeout_ns, abort_flag)))
+                    break;
+                mbar_arrive_expect_tx(bar_q, C::TILES * C::Q_TILE_BYTES);
+                for (int t = 0; t < C::TILES; ++t)
+                    for (int c = 0; c < C::KCH; ++c)
+                        tma_load_3d(smem + C::SMEM_Q + t * C::Q_TILE_BYTES + c * C::CHUNK_BYTES,
+                                    &tmQ, bar_q, c * 64, q_base + t * C::BM, bh);
+                for (int j = 0; j < nblk; ++j, ++g) {
+                    const int s = g % C::STAGES;
+                    const uint32_t ph = (g / C::STAGES) & 1;
+                    if (!(ok = mbar_wait(&bar_kempty[s], ph ^ 1, p.timeout_ns, abort_flag))) break;
+                    mbar_arrive_expect_tx(&bar_kfull[s], C::KV_TILE_BYTES);
+                    for (int c = 0; c < C::KCH; ++c)
+                        tma_load_3d(smem + C::SMEM_K + s * C::KV_TILE_BYTES + c * C::CHUNK_BYTES,
+                                    &tmK, &bar_kfull[s], c * 64, j * C::BN, bkv);
+                    ++gk;
+                    if (!(ok = mbar_wait(&bar_vempty[s], ph ^ 1, p.timeout_ns, abort_flag))) break;
+                    mbar_arrive_expect_tx(&bar_vfull[s], C::KV_TILE_BYTES);
+                    for (int c = 0; c < C::KCH; ++c)
+                        tma_load_3d(smem + C::SMEM_V + s * C::KV_TILE_BYTES + c * C::CHUNK_BYTES,
+                                    &tmV, &bar_vfull[s], c * 64, j * C::BN, bkv);
+                }
+            }
+            if (!ok) fail();
+            // Do not leave while our copies may still be landing in shared memory: the last
+            // STAGES K and V copies issued, and the last Q copy.
+            for (int j = max(0, gk - C::STAGES); j < gk; ++j)
+                mbar_wait_drain(&bar_kfull[j % C::STAGES], (j / C::STAGES) & 1, p.timeout_ns);
+            for (int j = max(0, g - C::STAGES); j < g; ++j)
+                mbar_wait_drain(&bar_vfull[j % C::STAGES], (j / C::STAGES) & 1, p.timeout_ns);
+            if (uc > 0 && !mbar_wait_drain(bar_q, (uc - 1) & 1, p.timeout_ns)) fail();
+        }
+    } else if (warp == 8) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idS = idesc_bf16(C::BM, C::BN, false, false);
+            constexpr uint32_t idPV = idesc_bf16(C::BM, D, false, true);
+            const uint32_t sQ = smem_u32(smem + C::SMEM_Q);
+            const uint32_t sK = smem_u32(smem + C::SMEM_K);
+            const uint32_t sV = smem_u32(smem + C::SMEM_V);
+            auto issue_S = [&](int t, int s) {
+                const uint32_t qa = sQ + t * C::Q_TILE_BYTES;
+                const uint32_t ka = sK + s * C::KV_TILE_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk / 4) * C::CHUNK_BYTES + (kk % 4) * 32;
+                    mma_ss(tmem + C::tm_s(t), sdesc_sw128(qa + off, 16, 1024),
+                           sdesc_sw128(ka + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+                }
+            };
+            constexpr int KK_PART = C::BN / 16 / C::P_PARTS;
+            auto issue_PV = [&](int t, int s, bool accumulate, int part) {
+                const uint32_t va = sV + s * C::KV_TILE_BYTES;
+#pragma unroll
+                for (int kk = part * KK_PART; kk < (part + 1) * KK_PART; ++kk)
+                    mma_ts(tmem + C::tm_o(t), tmem + C::tm_s(t) + kk * 8,
+                           sdesc_sw128(va + kk * 2048, C::CHUNK_BYTES, 1024), idPV,
+                           (accumulate || kk > 0) ? 1u : 0u);
+            };
+            // cb = key blocks consumed before this one (the P barriers' phase), the same for
+            // both tiles here; accumulate unless this is a unit's first block.
+            auto wait_issue_PV = [&](int t, int s, int cb, bool first) {
+#pragma unroll
+                for (int part = 0; part < C::P_PARTS; ++part) {
+                    uint64_t* bar = part + 1 < C::P_PARTS
+                                        ? &bar_ppart[t * (C::P_PARTS - 1) + part]
+                                        : &bar_pfull[t];
+                    if (!mbar_wait(bar, cb & 1, p.timeout_ns, abort_flag)) return false;
+                    tc_fence_after();
+                    issue_PV(t, s, !first || part > 0, part);
+                }
+                return true;
+            };
+            // Per unit: S_0(0) S_1(0), then per key block j: P V_0(j), S_0(j+1), P V_1(j),
+            // S_1(j+1); the commit after the unit's last score MMA releases the Q tiles.
+            bool ok = true;
+            int g = 0;   // ring position of the unit's block 0 (= blocks consumed so far)
+            int uc = 0;  // units started
+            for (int lin = blockIdx.x; ok && lin < n_units; lin += gridDim.x, ++uc) {
+                if (!(ok = mbar_wait(bar_q, uc & 1, p.timeout_ns, abort_flag))) break;
+                if (!(ok = mbar_wait(&bar_kfull[g % C::STAGES], (g / C::STAGES) & 1, p.timeout_ns,
+                                     abort_flag)))
+                    break;
+                tc_fence_after();
+                issue_S(0, g % C::STAGES);
+                tc_commit(&bar_sfull[0]);
+                issue_S(1, g % C::STAGES);
+                tc_commit(&bar_sfull[1]);
+                tc_commit(&bar_kempty[g % C::STAGES]);
+                if (nblk == 1) tc_commit(bar_qempty);
+                for (int j = 0; ok && j < nblk; ++j) {
+                    const int gj = g + j, gn = gj + 1;
+                    const int s = gj % C::STAGES, sn = gn % C::STAGES;
+                    const uint32_t ph = (gj / C::STAGES) & 1, phn = (gn / C::STAGES) & 1;
+                    if (!(ok = mbar_wait(&bar_vfull[s], ph, p.timeout_ns, abort_flag))) break;
+                    if (!(ok = wait_issue_PV(0, s, gj, j == 0))) break;
+                    tc_commit(&bar_ofull[0]);
+                    if (j + 1 < nblk) {
+                        if (!(ok = mbar_wait(&bar_kfull[sn], phn, p.timeout_ns, abort_flag))) break;
+                        tc_fence_after();
+                        issue_S(0, sn);
+                        tc_commit(&bar_sfull[0]);
+                    }
+                    if (!(ok = wait_issue_PV(1, s, gj, j == 0))) break;
+                    tc_commit(&bar_ofull[1]);
+                    tc_commit(&bar_vempty[s]);
+                    if (j + 1 < nblk) {
+                        issue_S(1, sn);
+                        tc_commit(&bar_sfull[1]);
+                        tc_commit(&bar_kempty[sn]);
+                        if (j + 2 == nblk) tc_commit(bar_qempty);
+                    }
+                }
+                g += nblk;
+            }
+            if (!ok) fail();
+            tc_commit(bar_done);
+            mbar_wait_drain(bar_done, 0, p.timeout_ns);
+        }
+      }
+    } else {
+        regs_increase<C::REGS_SOFTMAX_PERSIST>();
+        // ------------------------------------------------------------ softmax warpgroups
+        const int t = warp / 4;
+        const int r = threadIdx.x % C::BM;
+        const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
+        const uint32_t tS = tmem + lane_base + C::tm_s(t);
+        const uint32_t tO = tmem + lane_base + C::tm_o(t);
+        const float c = p.scale_log2;
+        const int lim = p.N;  // every key is visible
+        bool ok = true;
+        int cb = 0;  // key blocks processed (the phase of this tile's barriers)
+        for (int lin = blockIdx.x; ok && lin < n_units; lin += gridDim.x) {
+            float m = -INFINITY;  // running max of S * c (log2 units), possibly stale by <= 8
+            float l = 0.f;        // running sum of exp2(S * c - m)
+            for (int j = 0; j < nblk; ++j, ++cb) {
+                ok = mbar_wait(&bar_sfull[t], cb & 1, p.timeout_ns, abort_flag);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t s[C::BN];
+#pragma unroll
+                for (int q = 0; q < C::BN / 32; ++q) tmem_ld32(tS + q * 32, s + q * 32);
+                tmem_ld_wait();
+#pragma unroll
+                for (int q = 0; q < C::BN / 32; ++q) reg_fence32(s + q * 32);
+                const int k0 = j * C::BN;
+                if (k0 + C::BN > lim) {
+#pragma unroll
+                    for (int i = 0; i < C::BN; ++i)
+                        if (k0 + i >= lim) s[i] = __float_as_uint(-INFINITY);
+                }
+                float mx8[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) mx8[k] = __uint_as_float(s[k]);
+#pragma unroll
+                for (int i = 8; i < C::BN; i += 8)
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], __uint_as_float(s[i + k]));
+#pragma unroll
+                for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+                    for (int k = 0; k < w; ++k) mx8[k] = fmaxf(mx8[k], mx8[k + w]);
+                const float m_new = fmaxf(m, mx8[0] * c);
+                const bool grow = m_new > m + 8.0f;
+                const float alpha = (grow && m != -INFINITY) ? ex2(m - m_new) : 1.0f;
+                if (grow) {
+                    l *= alpha;
+                    m = m_new;
+                }
+                if (__any_sync(0xffffffffu, grow && j > 0)) {
+                    ok = mbar_wait(&bar_ofull[t], (cb - 1) & 1, p.timeout_ns, abort_flag);
+                    if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                    tc_fence_after();
+                    const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+                    for (int q = 0; q < D / 32; ++q) {
+                        uint32_t o[32];
+                        tmem_ld32(tO + q * 32, o);
+                        tmem_ld_wait();
+                        reg_fence32(o);
+#pragma unroll
+                        for (int i = 0; i < 32; i += 2) {
+                            const float2 y = fmul2(make_float2(__uint_as_float(o[i]),
+                                                               __uint_as_float(o[i + 1])), a2);
+                            o[i] = __float_as_uint(y.x);
+                            o[i + 1] = __float_as_uint(y.y);
+                        }
+                        tmem_st32(tO + q * 32, o);
+                    }
+                }
+                const float mb = (m == -INFINITY) ? 0.f : m;
+                const float2 c2 = make_float2(c, c);
+                const float2 nm2 = make_float2(-mb, -mb);
+                float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                                 make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                constexpr int WP = C::BN / 2 / C::P_PARTS;
+#pragma unroll
+                for (int part = 0; part < C::P_PARTS; ++part) {
+                    uint32_t pk[WP];
+#pragma unroll
+                    for (int i = 0; i < WP; ++i) {
+                        const int e0 = part * 2 * WP + 2 * i;
+                        const float2 x = ffma2(make_float2(__uint_as_float(s[e0]),
+                                                           __uint_as_float(s[e0 + 1])), c2, nm2);
+                        const float2 e = make_float2(ex2(x.x), ex2(x.y));
+                        acc[i % 4] = fadd2(acc[i % 4], e);
+                        pk[i] = pack_bf16x2(e.x, e.y);
+                    }
+                    if constexpr (WP == 32) tmem_st32(tS + part * WP, pk);
+                    else tmem_st16(tS + part * WP, pk);
+                    tmem_st_wait();
+                    tc_fence_before();
+                    mbar_arrive(part + 1 < C::P_PARTS ? &bar_ppart[t * (C::P_PARTS - 1) + part]
+                                                      : &bar_pfull[t]);
+                }
+                l += ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+                     ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+            }
+            // -------------------------------------------------------- epilogue of the unit
+            if (ok) ok = mbar_wait(&bar_ofull[t], (cb - 1) & 1, p.timeout_ns, abort_flag);
+            if (__all_sync(0xffffffffu, ok)) {
+                tc_fence_after();
+                const int lin_e = opaque(lin);  // recomputed here, not kept through the loop
+                const int bh = lin_e / nx;
+                const int row = (lin_e - bh * nx) * C::ROWS_PER_CTA + t * C::BM + r;
+                const float inv_l = l > 0.f ? 1.0f / l : 0.f;
+                const size_t o_off = ((size_t)bh * p.N + (row < p.N ? row : 0)) * D;
+                const bool in_range = row < p.N && in_bounds(p.err, o_off, D, p.dbg.q);
+                __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + o_off;
+#pragma unroll
+                for (int q = 0; q < D / 32; ++q) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + q * 32, o);
+                    tmem_ld_wait();
+                    reg_fence32(o);
+                    uint32_t w[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l,
+                                           __uint_as_float(o[2 * i + 1]) * inv_l);
+                    if (in_range) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                    }
+                }
+                const size_t l_off = (size_t)bh * p.N + row;
+                if (in_range && in_bounds(p.err, l_off, 1, p.dbg.lse))
+                    p.lse[l_off] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+            } else {
+                fail();
+                ok = false;
+            }
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 8) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+
 template <int D, bool PACKED>
 cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                         const FwdParams& p, int B, cudaStream_t stream) {
+                         const FwdParams& p, int B, int num_sms, cudaStream_t stream) {
     using C = FwdCfg<D>;
     static std::atomic<uint64_t> configured{0};  // one bit per device
     if (cudaError_t e = set_smem_limit_once(configured, C::SMEM_BYTES,
                                             fa_fwd_kernel<D, PACKED, false>,
-                                            fa_fwd_kernel<D, PACKED, !PACKED>);
+                                            fa_fwd_kernel<D, PACKED, !PACKED>,
+                                            fa_fwd_persist_kernel<D>);
         e != cudaSuccess)
         return e;
-    dim3 grid((p.N + C::ROWS_PER_CTA - 1) / C::ROWS_PER_CTA, p.H, B);
+    const int nx = (p.N + C::ROWS_PER_CTA - 1) / C::ROWS_PER_CTA;
+    const long long units = (long long)nx * p.H * B;
+    // Units of equal cost (head-major, no causal mask, no key lengths) and more of them than
+    // SMs: the persistent kernel, one CTA per SM.  Otherwise one CTA per unit in the
+    // heaviest-first order, which the hardware's CTA scheduler balances better than a static
+    // assignment when units differ in cost.
+    if (!PACKED && !p.causal && p.seqlens == nullptr && units > num_sms) {
+        fa_fwd_persist_kernel<D><<<num_sms, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+        return cudaGetLastError();
+    }
+    dim3 grid(nx, p.H, B);
     // Head-major causal launches take the grouped heaviest-first order (its own instantiation,
     // so that the other launches keep their code unchanged).
     if (!PACKED && p.causal)
@@ -516,13 +892,12 @@ cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 
 cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const FwdParams& p, int B, int num_sms, cudaStream_t stream) {
-    (void)num_sms;
     const bool packed = p.cu_seqlens != nullptr;
     if (d == 64)
-        return packed ? launch_fwd_d<64, true>(tq, tk, tv, p, B, stream)
-                      : launch_fwd_d<64, false>(tq, tk, tv, p, B, stream);
-    return packed ? launch_fwd_d<128, true>(tq, tk, tv, p, B, stream)
-                  : launch_fwd_d<128, false>(tq, tk, tv, p, B, stream);
+        return packed ? launch_fwd_d<64, true>(tq, tk, tv, p, B, num_sms, stream)
+                      : launch_fwd_d<64, false>(tq, tk, tv, p, B, num_sms, stream);
+    return packed ? launch_fwd_d<128, true>(tq, tk, tv, p, B, num_sms, stream)
+                  : launch_fwd_d<128, false>(tq, tk, tv, p, B, num_sms, stream);
 }
 
 }  // namespace fa

@@ -378,26 +378,5 @@ __device__ __forceinline__ uint32_t pack_bf16x2_alu(float lo, float hi) {
     return __byte_perm(a, b, 0x7632);  // high halves: a -> bits 0-15, b -> bits 16-31
 }
 
-// 2^x for two values on the FMA pipe (no MUFU), for splitting exponentials between the two
-// units.  Cody-Waite style range reduction x = n + f, n = round-to-nearest(x) obtained with the
-// 1.5 * 2^23 shift (the sum's low mantissa bits hold n), f in [-1/2, 1/2]; 2^f from a degree-3
-// polynomial with minimax relative error 7.5e-5 on that interval (coefficients fitted here by a
-// Remez exchange, rounded to fp32); 2^n applied by adding n to the exponent field.  Results for
-// x < -125 are 0, like the flush-to-zero MUFU path; x must be < 128.
-__device__ __forceinline__ float2 exp2_fma2(float2 x) {
-    const float2 shift = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
-    const float2 t = fadd2(x, shift);                            // n in the low mantissa bits
-    const float2 n = fadd2(t, make_float2(-12582912.0f, -12582912.0f));
-    const float2 f = fadd2(x, make_float2(-n.x, -n.y));
-    float2 q = ffma2(make_float2(0.0551716685f, 0.0551716685f), f,
-                     make_float2(0.2426111251f, 0.2426111251f));
-    q = ffma2(q, f, make_float2(0.6932609677f, 0.6932609677f));
-    q = ffma2(q, f, make_float2(0.9999280572f, 0.9999280572f));
-    // (bits(t) << 23) == n << 23: the shift's own bits sit above bit 8 and shift out.
-    const int ex = __float_as_int(q.x) + (__float_as_int(t.x) << 23);
-    const int ey = __float_as_int(q.y) + (__float_as_int(t.y) << 23);
-    return make_float2(x.x < -125.0f ? 0.f : __int_as_float(ex), x.y < -125.0f ? 0.f : __int_as_float(ey));
-}
-
 }  // namespace sm100
 }  // namespace fa
