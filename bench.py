@@ -116,12 +116,29 @@ def load_peaks() -> tuple[dict, str]:
 
 KERNEL_SOURCES = {
     "fa_fwd_kernel": ("fa_fwd.cu", "sm100.cuh", "fa_internal.h"),
+    "fa_fwd_persist_kernel": ("fa_fwd.cu", "sm100.cuh", "fa_internal.h"),
     "fa_bwd_kernel": ("fa_bwd.cu", "fa_bwd_common.cuh", "sm100.cuh", "fa_internal.h"),
+    "fa_bwd_persist_kernel": ("fa_bwd.cu", "fa_bwd_common.cuh", "sm100.cuh", "fa_internal.h"),
     "fa_fwd_d256_kernel": ("fa_fwd_d256.cu", "sm100.cuh", "fa_internal.h"),
     "fa_fwd_fp8_kernel": ("fa_fwd_fp8.cu", "fa_fwd_fp8.h", "sm100.cuh", "fa_internal.h"),
     "fa_bwd_d256_kernel": ("fa_bwd_d256.cu", "fa_bwd_common.cuh", "sm100.cuh", "fa_internal.h"),
     "fa_decode_kernel": ("fa_decode.cu", "fa_decode.h", "sm100.cuh", "fa_internal.h"),
 }
+
+
+def main_kernels(w: workloads.Workload, num_sms: int) -> tuple[str, str]:
+    """Names of the fused forward and backward kernels the library launches for `w`: the
+    persistent ones when every work unit costs the same (no causal mask, no key lengths) and
+    there are more units than SMs, the one-CTA-per-unit ones otherwise."""
+    equal = not w.causal and w.pad_range is None
+    fwd_units = -(-w.N // 256) * w.H * w.B
+    bwd_units = -(-w.N // 128) * w.kv_heads * w.B
+    steps = (w.H // w.kv_heads) * -(-w.N // 128)  # query steps of one backward unit
+    fwd = ("fa_fwd_persist_kernel" if equal and fwd_units > num_sms and -(-w.N // 128) <= 32
+           else "fa_fwd_kernel")
+    bwd = ("fa_bwd_persist_kernel" if equal and bwd_units > num_sms and steps <= 16
+           else "fa_bwd_kernel")
+    return fwd, bwd
 
 
 def kernel_source_hash(kernel: str) -> str:
@@ -393,7 +410,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
     clock_summary = clocks.summary()
     timed_s = elapsed_ms * 1e-3
     wname = args.workload
-    traffic = dram_traffic("fa_bwd_kernel", wname)
+    fwd_name, bwd_name = main_kernels(w, torch.cuda.get_device_properties(dev).multi_processor_count)
+    traffic = dram_traffic(bwd_name, wname)
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -419,12 +437,12 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> dict | None:
                    "fwd_pct_of_2250": round(100 * fwd_tflops / NOMINAL_PEAK_TFLOPS, 2),
                    "bwd_pct_of_2250": round(100 * bwd_tflops / NOMINAL_PEAK_TFLOPS, 2),
                    "step_ms_p10_p50_p90": [round(_pct(step_ms, q), 4) for q in (10, 50, 90)]},
-        "roofline": roofline_tensor("fa_bwd_kernel (fused backward: all five backward GEMMs)",
+        "roofline": roofline_tensor(f"{bwd_name} (fused backward: all five backward GEMMs)",
                                     bwd_kernel_tflops, bwd_kernel_ms, peaks, peak_src, timed_s,
                                     clock_summary, traffic),
-        "roofline_fwd": roofline_tensor("fa_fwd_kernel", fwd_kernel_tflops, fwd_kernel_ms, peaks,
+        "roofline_fwd": roofline_tensor(fwd_name, fwd_kernel_tflops, fwd_kernel_ms, peaks,
                                         peak_src, timed_s, clock_summary,
-                                        dram_traffic("fa_fwd_kernel", wname)),
+                                        dram_traffic(fwd_name, wname)),
         "e2e": {"value": round(step_flops * e2e_steps * world / (max(e2e_ms, 1e-9) * 1e-3) / 1e12, 2),
                 "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps, "copies": "pinned host memory, own streams, overlapped "

@@ -199,6 +199,7 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
     p.cu_seqlens = cu_seqlens;
     p.T = T;
     p.err = dev->err_flag;
+    p.B = B;
     p.H = H;
     p.N = N;
     p.H_kv = H_kv;
@@ -377,6 +378,7 @@ static fa_status bwd_impl(const void* q, const void* k, const void* v, const voi
     p.causal = causal ? 1 : 0;
     p.timeout_ns = g_timeout_ns.load();
     const bool packed = cu_seqlens != nullptr;
+    p.num_sms = dev->num_sms;
     p.dbg = extents(B, H, H_kv, N, d, T, packed);
 
     CUtensorMap tq, tk, tv, tdo;

@@ -29,6 +29,7 @@ static __device__ __align__(256) unsigned char g_bwd_scratch[kScratchBytes];
 struct ScratchDevice {
     bool ready = false;      // set-up done for this device
     bool supported = false;  // compute capability 10.0
+    int num_sms = 0;         // multiprocessors (the backward's persistent grid)
     void* scratch = nullptr; // device address of g_bwd_scratch on this device
 };
 ScratchDevice g_scratch_dev[kMaxDevices];
@@ -36,7 +37,7 @@ std::mutex g_scratch_mutex;
 
 // One-time set-up for the current device: check it is a B200-class GPU and look up the
 // device address of the scratch array.  Allocates nothing.
-fa_status scratch_for_current_device(void** out) {
+fa_status scratch_for_current_device(void** out, int* num_sms) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_scratch_mutex);
@@ -44,7 +45,8 @@ fa_status scratch_for_current_device(void** out) {
     if (!s.ready) {
         int major = 0, minor = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&s.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return FA_ERR_CUDA;
         s.supported = (major == 10 && minor == 0);
         if (s.supported) {
@@ -64,6 +66,7 @@ fa_status scratch_for_current_device(void** out) {
     }
     if (!s.supported) return FA_ERR_UNSUPPORTED;
     *out = s.scratch;
+    *num_sms = s.num_sms;
     return FA_OK;
 }
 
@@ -90,7 +93,8 @@ extern "C" FA_API fa_status fa_bwd_noalloc(const void* q, const void* k, const v
     // Larger problems than the fixed scratch holds are refused, never truncated.
     if (need > kScratchBytes) return FA_ERR_WORKSPACE;
     void* scratch = nullptr;
-    fa_status st = scratch_for_current_device(&scratch);
+    int num_sms = 0;
+    fa_status st = scratch_for_current_device(&scratch, &num_sms);
     if (st != FA_OK) return st;
 
     // Carve the scratch exactly as fa_bwd carves its workspace.  Nothing in it has to start
@@ -129,6 +133,7 @@ extern "C" FA_API fa_status fa_bwd_noalloc(const void* q, const void* k, const v
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
     p.timeout_ns = fa::wait_timeout_ns();
+    p.num_sms = num_sms;
     p.dbg = fa::extents(B, H, H, N, d, 0, false);
 
     CUtensorMap tq, tk, tv, tdo;

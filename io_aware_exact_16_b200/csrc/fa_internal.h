@@ -60,7 +60,7 @@ struct FwdParams {
     const int* cu_seqlens; // device int32 [B + 1] packed sequence offsets or nullptr
     int T;                 // packed: rows of the packed tensors
     int* err;              // device error flag
-    int H, N;
+    int B, H, N;
     int H_kv;              // key/value heads; query head h reads K/V head h / (H / H_kv)
     float scale_log2;      // scale * log2(e)
     int causal;
@@ -91,6 +91,7 @@ struct BwdParams {
     float scale_log2;
     int causal;
     uint64_t timeout_ns;
+    int num_sms;           // SMs of the device (the persistent grid); 0: one CTA per key block
     Extents dbg;
 };
 

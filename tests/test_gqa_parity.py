@@ -35,6 +35,9 @@ SHAPES = [
     # causal launches walk groups of 16 heads: B*H_kv = 21 is one full group and a partial one
     (3, 14, 7, 300, 128, True, None),
     (3, 14, 7, 300, 64, True, None),
+    # more units than SMs, non-causal, 16 query steps per key block: the persistent forward
+    # and backward kernels with two query heads per key/value head
+    (4, 32, 16, 1024, 128, False, None),
 ]
 
 
