@@ -152,15 +152,17 @@ def kernel_source_hash(kernel: str) -> str:
 
 
 def dram_traffic(kernel: str, workload: str) -> float | None:
-    """Per-launch DRAM bytes from the committed ncu summary, or None when it is stale."""
+    """Per-launch DRAM bytes of `kernel` at `workload` from the committed ncu summaries
+    (profiles/traffic.json, keyed "kernel @ workload"), or None when the kernel's sources have
+    changed since the counters were taken."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             data = json.load(f)
     except (OSError, ValueError):
         return None
-    entry = data.get(kernel, {})
-    if entry.get("workload") != workload or entry.get("source_hash") != kernel_source_hash(kernel):
+    entry = data.get(f"{kernel} @ {workload}", {})
+    if entry.get("source_hash") != kernel_source_hash(kernel):
         return None
     return float(entry["dram_bytes_per_launch"])
 
