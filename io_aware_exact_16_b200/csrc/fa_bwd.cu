@@ -99,6 +99,18 @@ struct BwdCfg {
     static constexpr uint32_t REGS_COMPUTE_PERSIST = 128, REGS_OTHER_PERSIST = 104;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t TM_A = 0, TM_B = 128, TM_DV = 256, TM_DK = 256 + D;
+    // Warpgroup h reads the fp32 S^T / dP^T columns [64h, 64h + 64) of its region and writes
+    // the bf16 P^T / dS^T of its 64 queries (32 columns) back into the first half of those
+    // same columns, so no warpgroup overwrites columns the other still reads.  The MMAs that
+    // read P^T / dS^T as their A operand address each 16-query K step where it lies.
+#ifndef FA_BWD_OWN_COLUMNS
+#define FA_BWD_OWN_COLUMNS 1
+#endif
+    static constexpr bool OWN_COLUMNS = FA_BWD_OWN_COLUMNS;
+    __device__ static constexpr uint32_t bf16_col(int h) { return OWN_COLUMNS ? 64u * h : 32u * h; }
+    __device__ static constexpr uint32_t a_col(int kk) {
+        return OWN_COLUMNS ? (uint32_t)((kk / 4) * 64 + (kk % 4) * 8) : (uint32_t)(kk * 8);
+    }
 };
 
 // ---------------------------------------------------------------------------- main kernel
@@ -398,7 +410,7 @@ __global__ void __launch_bounds__(512, 1)
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < C::BM / 16; ++kk)
-                mma_ts(tmem + C::TM_DV, tmem + C::TM_A + kk * 8, dDO_mn + mnmaj(kk), idKV,
+                mma_ts(tmem + C::TM_DV, tmem + C::TM_A + C::a_col(kk), dDO_mn + mnmaj(kk), idKV,
                        (it > 0 || kk > 0) ? 1u : 0u);
             if (it + 1 < n_it) {
                 const int s1 = (it + 1) % C::QST;
@@ -413,7 +425,7 @@ __global__ void __launch_bounds__(512, 1)
                 // dK += dS^T Q, same shapes as dV (A = dS^T in tensor memory).
 #pragma unroll
                 for (int kk = 0; kk < C::BM / 16; ++kk)
-                    mma_ts(tmem + C::TM_DK, tmem + C::TM_B + kk * 8, dQ_mn + mnmaj(kk), idKV,
+                    mma_ts(tmem + C::TM_DK, tmem + C::TM_B + C::a_col(kk), dQ_mn + mnmaj(kk), idKV,
                            (it > 0 || kk > 0) ? 1u : 0u);
                 tc_commit(&bar_qempty[s]);
             }
@@ -536,12 +548,13 @@ __global__ void __launch_bounds__(512, 1)
                         if (key_padded || r > 64 * h + e) P[e] = 0.f;
                 }
             }
-            named_barrier(1, 256);  // every S^T column read before P^T overwrites columns
+            // (shared columns only) every S^T column read before P^T overwrites columns
+            if constexpr (!C::OWN_COLUMNS) named_barrier(1, 256);
             if (ok) {
                 uint32_t pw[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) pw[e] = pack_bf16x2(P[2 * e], P[2 * e + 1]);
-                tmem_st32(tmem + lane_base + C::TM_A + 32 * h, pw);
+                tmem_st32(tmem + lane_base + C::TM_A + C::bf16_col(h), pw);
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(bar_pfull);
@@ -573,14 +586,14 @@ __global__ void __launch_bounds__(512, 1)
                     }
                 }
             }
-            // Next block's lse / D into the other buffer: every thread has passed this
-            // iteration's first barrier, so nobody still reads that buffer, and the barrier
-            // below orders these stores before the next iteration's reads.
+            // Next block's lse / D into the other buffer.  Its last reads were in the previous
+            // iteration, before every thread passed that iteration's barrier below, and the
+            // barrier below orders these stores before the next iteration's reads.
             if (it + 1 < n_it) store_vectors(it + 1);
-            named_barrier(1, 256);  // every dP^T column read before dS^T overwrites columns
+            named_barrier(1, 256);  // next step's lse / D stored; shared columns: dP^T read
             if (ok) {
                 // d = 128: dK reads dS^T from tensor memory; d = 64 reads the shared tile below.
-                if constexpr (D == 128) tmem_st32(tmem + lane_base + C::TM_B + 32 * h, dw);
+                if constexpr (D == 128) tmem_st32(tmem + lane_base + C::TM_B + C::bf16_col(h), dw);
                 // dS^T row r, queries [64h, 64h+64) = one 128-byte row of query chunk h; 16-byte
                 // unit u sits at position u ^ (r % 8) (the 128-byte swizzle the MMA reads).
 #pragma unroll
@@ -912,7 +925,7 @@ __global__ void __launch_bounds__(512, 1)
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < C::BM / 16; ++kk)
-                    mma_ts(tmem + C::TM_DV, tmem + C::TM_A + kk * 8, dDO_mn + mnmaj(kk), idKV,
+                    mma_ts(tmem + C::TM_DV, tmem + C::TM_A + C::a_col(kk), dDO_mn + mnmaj(kk), idKV,
                            (it > 0 || kk > 0) ? 1u : 0u);
                 if (it + 1 < n_it) {
                     if (!(ok = mbar_wait(&bar_qfull[(g + 1) % C::QST], ((g + 1) / C::QST) & 1,
@@ -926,7 +939,7 @@ __global__ void __launch_bounds__(512, 1)
                 if constexpr (D == 128) {
 #pragma unroll
                     for (int kk = 0; kk < C::BM / 16; ++kk)
-                        mma_ts(tmem + C::TM_DK, tmem + C::TM_B + kk * 8, dQ_mn + mnmaj(kk), idKV,
+                        mma_ts(tmem + C::TM_DK, tmem + C::TM_B + C::a_col(kk), dQ_mn + mnmaj(kk), idKV,
                                (it > 0 || kk > 0) ? 1u : 0u);
                     tc_commit(&bar_qempty[s]);
 #pragma unroll
@@ -1030,12 +1043,13 @@ __global__ void __launch_bounds__(512, 1)
                         for (int e = 0; e < 64; ++e) P[e] = 0.f;
                     }
                 }
-                named_barrier(1, 256);  // every S^T column read before P^T overwrites columns
+                // (shared columns only) every S^T column read before P^T overwrites columns
+                if constexpr (!C::OWN_COLUMNS) named_barrier(1, 256);
                 if (ok) {
                     uint32_t pw[32];
 #pragma unroll
                     for (int e = 0; e < 32; ++e) pw[e] = pack_bf16x2(P[2 * e], P[2 * e + 1]);
-                    tmem_st32(tmem + lane_base + C::TM_A + 32 * h, pw);
+                    tmem_st32(tmem + lane_base + C::TM_A + C::bf16_col(h), pw);
                     tmem_st_wait();
                     tc_fence_before();
                     mbar_arrive(bar_pfull);
@@ -1068,9 +1082,9 @@ __global__ void __launch_bounds__(512, 1)
                     }
                 }
                 if (it + 1 < n_it) store_vectors(g + 1);
-                named_barrier(1, 256);  // every dP^T column read before dS^T overwrites columns
+                named_barrier(1, 256);  // next step's lse / D stored; shared columns: dP^T read
                 if (ok) {
-                    if constexpr (D == 128) tmem_st32(tmem + lane_base + C::TM_B + 32 * h, dw);
+                    if constexpr (D == 128) tmem_st32(tmem + lane_base + C::TM_B + C::bf16_col(h), dw);
 #pragma unroll
                     for (int v4 = 0; v4 < 8; ++v4)
                         *reinterpret_cast<uint4*>(ds_row + ((v4 ^ sw) << 4)) =
