@@ -98,6 +98,7 @@ struct BwdCfg {
     // 88 registers: 2 x 128 + 104 + 152 there.
     static constexpr uint32_t REGS_COMPUTE_PERSIST = 128, REGS_OTHER_PERSIST = 104;
     static constexpr uint32_t TMEM_COLS = 512;
+
     static constexpr uint32_t TM_A = 0, TM_B = 128, TM_DV = 256, TM_DK = 256 + D;
     // Warpgroup h reads the fp32 S^T / dP^T columns [64h, 64h + 64) of its region and writes
     // the bf16 P^T / dS^T of its 64 queries (32 columns) back into the first half of those
@@ -255,25 +256,32 @@ __global__ void __launch_bounds__(512, 1)
         // Named barriers have no timeout: every drain thread executes each of them, also after
         // a failed wait (`ok` then only skips the work).
         bool ok = true;
+        // ||dO|| of query row r of step s, or -1 for rows past the sequence (scale 0).  Loaded
+        // one step ahead, so its latency overlaps the previous step's reductions.
+        auto load_norm = [&](Step s) -> float {
+            const int q = q_block(s) * C::BM + r;
+            return q < ext.Lq && in_bounds(p.err, (size_t)q_head(s) * p.N + q, 1, p.dbg.vec)
+                       ? p.dOnorm[(size_t)q_head(s) * p.N + q] : -1.f;
+        };
         Step st{0, 0};
+        float norm = load_norm(st);
         for (int it = 0; it < n_it; ++it, st = next_step(st)) {
             const int q0 = q_block(st) * C::BM;
-            // fixed-point scale of query q0 + r (rows past N: scale 0), shared by the drain
-            // warps; barrier 2 before the reads and again after the last read of the step
-            {
-                const int q = q0 + r;
-                // (-1, a bound beyond fp32 range, adds nothing; the dQ conversion reports it)
-                s_scale[r] = q < ext.Lq && in_bounds(p.err, (size_t)q_head(st) * p.N + q, 1, p.dbg.vec)
-                                 ? fmaxf(fixed_point_scale(p.dOnorm[(size_t)q_head(st) * p.N + q], factor), 0.f)
-                                 : 0.f;
-            }
+            // fixed-point scale of query q0 + r, shared by the drain warps; barrier 2 before the
+            // reads and again after the last read of the step.  (A non-finite norm or bound
+            // gives -1, which adds nothing; the dQ conversion reports it.)
+            s_scale[r] = norm >= 0.f ? fmaxf(fixed_point_scale(norm, factor), 0.f) : 0.f;
+            if (it + 1 < n_it) norm = load_norm(next_step(st));
             named_barrier(2, 128);
             const float* sc = s_scale;
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_dqfull, it & 1, p.timeout_ns, abort_flag));
+            constexpr int NV = (D == 128) ? 128 : 64;
+            uint32_t v[NV];
+            int* acc = p.dq_acc + ((size_t)q_head(st) * p.N_pad + q0) * D;
+            const bool acc_ok = in_bounds(p.err, ((size_t)q_head(st) * p.N_pad + q0) * D,
+                                          (size_t)C::BM * D, p.dbg.acc);
             if (ok) {
                 tc_fence_after();
-                constexpr int NV = (D == 128) ? 128 : 64;
-                uint32_t v[NV];
 #pragma unroll
                 for (int q = 0; q < NV / 32; ++q) tmem_ld32(tmem + lane_base + C::TM_B + 32 * q, v + 32 * q);
                 tmem_ld_wait();
@@ -281,9 +289,7 @@ __global__ void __launch_bounds__(512, 1)
                 for (int q = 0; q < NV / 32; ++q) reg_fence32(v + 32 * q);
                 tc_fence_before();
                 mbar_arrive(bar_dqempty);           // B may take the next dP^T
-                int* acc = p.dq_acc + ((size_t)q_head(st) * p.N_pad + q0) * D;
-                if (in_bounds(p.err, ((size_t)q_head(st) * p.N_pad + q0) * D, (size_t)C::BM * D,
-                              p.dbg.acc)) {
+                if (acc_ok) {
                     if constexpr (D == 128) {
                         // dQ^T: lane = feature r, column = query e; a warp instruction covers 32
                         // consecutive features of one query row: one 128-byte line.
@@ -764,23 +770,30 @@ __global__ void __launch_bounds__(512, 1)
         for (int lin = blockIdx.x; lin < n_units; lin += gridDim.x, gs += n_it) {
             const Unit u = unit(lin);
             const float factor = head_bound_factor(p, u.bhk);
+            // ||dO|| of query row r of step s (-1 past N: scale 0), loaded one step ahead
+            auto load_norm = [&](Step s) -> float {
+                const int q = q_block(u, s) * C::BM + r;
+                const int qh = u.bh_first + s.g;
+                return q < p.N && in_bounds(p.err, (size_t)qh * p.N + q, 1, p.dbg.vec)
+                           ? p.dOnorm[(size_t)qh * p.N + q] : -1.f;
+            };
             Step st{0, 0};
+            float norm = load_norm(st);
             for (int it = 0; it < n_it; ++it, st = next_step(st)) {
                 const int q0 = q_block(u, st) * C::BM;
                 const int qh = u.bh_first + st.g;
-                {
-                    const int q = q0 + r;
-                    s_scale[r] = q < p.N && in_bounds(p.err, (size_t)qh * p.N + q, 1, p.dbg.vec)
-                                     ? fmaxf(fixed_point_scale(p.dOnorm[(size_t)qh * p.N + q], factor), 0.f)
-                                     : 0.f;
-                }
+                s_scale[r] = norm >= 0.f ? fmaxf(fixed_point_scale(norm, factor), 0.f) : 0.f;
+                if (it + 1 < n_it) norm = load_norm(next_step(st));
                 named_barrier(2, 128);
                 const float* sc = s_scale;
                 if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_dqfull, (gs + it) & 1, p.timeout_ns, abort_flag));
+                constexpr int NV = (D == 128) ? 128 : 64;
+                uint32_t v[NV];
+                int* acc = p.dq_acc + ((size_t)qh * p.N_pad + q0) * D;
+                const bool acc_ok =
+                    in_bounds(p.err, ((size_t)qh * p.N_pad + q0) * D, (size_t)C::BM * D, p.dbg.acc);
                 if (ok) {
                     tc_fence_after();
-                    constexpr int NV = (D == 128) ? 128 : 64;
-                    uint32_t v[NV];
 #pragma unroll
                     for (int q = 0; q < NV / 32; ++q) tmem_ld32(tmem + lane_base + C::TM_B + 32 * q, v + 32 * q);
                     tmem_ld_wait();
@@ -788,8 +801,7 @@ __global__ void __launch_bounds__(512, 1)
                     for (int q = 0; q < NV / 32; ++q) reg_fence32(v + 32 * q);
                     tc_fence_before();
                     mbar_arrive(bar_dqempty);  // B may take the next dP^T
-                    int* acc = p.dq_acc + ((size_t)qh * p.N_pad + q0) * D;
-                    if (in_bounds(p.err, ((size_t)qh * p.N_pad + q0) * D, (size_t)C::BM * D, p.dbg.acc)) {
+                    if (acc_ok) {
                         if constexpr (D == 128) {
 #pragma unroll
                             for (int e = 0; e < 128; e += 2) {
