@@ -65,6 +65,11 @@ struct Bwd256 {
     static constexpr uint32_t REGS_COMPUTE = 136, REGS_OTHER = 88, REGS_DRAIN = 152;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t TM_A = 0, TM_B = 64, TM_DQ = 128, TM_DV = 256, TM_DK = 384;
+    // Warpgroup h reads the fp32 S^T / dP^T columns [32h, 32h + 32) and writes the bf16 P^T /
+    // dS^T of its 32 queries (16 columns) into the first half of those same columns, so neither
+    // warpgroup overwrites columns the other still reads; the MMAs reading P^T / dS^T as A
+    // address each 16-query K step where it lies.
+    __device__ static constexpr uint32_t a_col(int kk) { return (uint32_t)((kk / 2) * 32 + (kk % 2) * 8); }
     static_assert(SMEM_BYTES <= 232448, "shared memory over the sm_100 per-CTA limit");
     static_assert(SMEM_DS % 1024 == 0 && SMEM_Q % 1024 == 0 && SMEM_DO % 1024 == 0,
                   "swizzled tiles must start on 1024-byte boundaries");
@@ -303,14 +308,14 @@ __global__ void __launch_bounds__(512, 1)
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < C::BM / 16; ++kk)
-                mma_ts(tmem + C::TM_DV, tmem + C::TM_A + kk * 8, dDOh_mn + mnmaj(kk), idKV,
+                mma_ts(tmem + C::TM_DV, tmem + C::TM_A + C::a_col(kk), dDOh_mn + mnmaj(kk), idKV,
                        (it > 0 || kk > 0) ? 1u : 0u);
             // dK[:, half] += dS^T Q[:, half]; after it nothing reads this step's Q and dO.
             if (!(ok = mbar_wait(bar_dsfull, it & 1, p.timeout_ns, abort_flag))) break;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < C::BM / 16; ++kk)
-                mma_ts(tmem + C::TM_DK, tmem + C::TM_B + kk * 8, dQh_mn + mnmaj(kk), idKV,
+                mma_ts(tmem + C::TM_DK, tmem + C::TM_B + C::a_col(kk), dQh_mn + mnmaj(kk), idKV,
                        (it > 0 || kk > 0) ? 1u : 0u);
             tc_commit(bar_qempty);
             // dQ^T[half] = K[:, half]^T dS^T (K = 128 keys), once the drain has copied the
@@ -406,12 +411,11 @@ __global__ void __launch_bounds__(512, 1)
                         if (key_padded || kidx > q0 + 32 * h + e) P[e] = 0.f;
                 }
             }
-            named_barrier(1, 256);  // every S^T column read before P^T overwrites columns
             if (ok) {
                 uint32_t pw[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) pw[e] = pack_bf16x2(P[2 * e], P[2 * e + 1]);
-                tmem_st16(tmem + lane_base + C::TM_A + 16 * h, pw);
+                tmem_st16(tmem + lane_base + C::TM_A + 32 * h, pw);
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(bar_pfull);
@@ -439,13 +443,13 @@ __global__ void __launch_bounds__(512, 1)
                     dw[e / 2 + 1] = pack_bf16x2(bq.x, bq.y);
                 }
             }
-            // Next step's lse / D into the other buffer: every thread has passed this step's
-            // first barrier, so nobody still reads that buffer, and the barrier below orders
-            // these stores before the next step's reads.
+            // Next step's lse / D into the other buffer.  Its last reads were in the previous
+            // step, before every thread passed that step's barrier below, and the barrier below
+            // orders these stores before the next step's reads.
             if (it + 1 < n_it) store_vectors(it + 1);
-            named_barrier(1, 256);  // every dP^T column read before dS^T overwrites columns
+            named_barrier(1, 256);  // the next step's lse / D stored
             if (ok) {
-                tmem_st16(tmem + lane_base + C::TM_B + 16 * h, dw);  // A of dK
+                tmem_st16(tmem + lane_base + C::TM_B + 32 * h, dw);  // A of dK
                 // dS^T row r, queries [32h, 32h+32): 16-byte units 4h..4h+3 of the row's 128
                 // bytes, unit u at position u ^ (r % 8) (the 128-byte swizzle the MMA reads).
                 // The dQ^T MMA of the previous step has finished reading the tile: dP^T of
