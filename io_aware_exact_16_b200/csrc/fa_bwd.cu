@@ -294,11 +294,14 @@ __global__ void __launch_bounds__(512, 1)
                         // dQ^T: lane = feature r, column = query e; a warp instruction covers 32
                         // consecutive features of one query row: one 128-byte line.
 #pragma unroll
-                        for (int e = 0; e < 128; e += 2) {
-                            const int2 x = to_fixed2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
-                                                     sc[e], sc[e + 1]);
+                        for (int e = 0; e < 128; e += 4) {
+                            const float4 s4 = *reinterpret_cast<const float4*>(sc + e);  // one shared load
+                            const int2 x = to_fixed2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]), s4.x, s4.y);
+                            const int2 y = to_fixed2(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]), s4.z, s4.w);
                             red_add_s32(acc + (size_t)e * D + r, x.x);
                             red_add_s32(acc + (size_t)(e + 1) * D + r, x.y);
+                            red_add_s32(acc + (size_t)(e + 2) * D + r, y.x);
+                            red_add_s32(acc + (size_t)(e + 3) * D + r, y.y);
                         }
                     } else {
                         // dQ: lane = query r, 64 features.  Convert, transpose 32 x 32 through
@@ -804,11 +807,14 @@ __global__ void __launch_bounds__(512, 1)
                     if (acc_ok) {
                         if constexpr (D == 128) {
 #pragma unroll
-                            for (int e = 0; e < 128; e += 2) {
-                                const int2 x = to_fixed2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
-                                                         sc[e], sc[e + 1]);
+                            for (int e = 0; e < 128; e += 4) {
+                                const float4 s4 = *reinterpret_cast<const float4*>(sc + e);  // one shared load
+                                const int2 x = to_fixed2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]), s4.x, s4.y);
+                                const int2 y = to_fixed2(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]), s4.z, s4.w);
                                 red_add_s32(acc + (size_t)e * D + r, x.x);
                                 red_add_s32(acc + (size_t)(e + 1) * D + r, x.y);
+                                red_add_s32(acc + (size_t)(e + 2) * D + r, y.x);
+                                red_add_s32(acc + (size_t)(e + 3) * D + r, y.y);
                             }
                         } else {
                             int* xp = reinterpret_cast<int*>(smem + C::SMEM_XPOSE) + (warp % 4) * 32 * 33;
