@@ -100,17 +100,17 @@ struct BwdCfg {
     static constexpr uint32_t TMEM_COLS = 512;
 
     static constexpr uint32_t TM_A = 0, TM_B = 128, TM_DV = 256, TM_DK = 256 + D;
-    // Warpgroup h reads the fp32 S^T / dP^T columns [64h, 64h + 64) of its region and writes
-    // the bf16 P^T / dS^T of its 64 queries (32 columns) back into the first half of those
-    // same columns, so no warpgroup overwrites columns the other still reads.  The MMAs that
-    // read P^T / dS^T as their A operand address each 16-query K step where it lies.
-#ifndef FA_BWD_OWN_COLUMNS
-#define FA_BWD_OWN_COLUMNS 1
-#endif
-    static constexpr bool OWN_COLUMNS = FA_BWD_OWN_COLUMNS;
-    __device__ static constexpr uint32_t bf16_col(int h) { return OWN_COLUMNS ? 64u * h : 32u * h; }
-    __device__ static constexpr uint32_t a_col(int kk) {
-        return OWN_COLUMNS ? (uint32_t)((kk / 4) * 64 + (kk % 4) * 8) : (uint32_t)(kk * 8);
+    // Own columns: warpgroup h reads the fp32 S^T / dP^T columns [64h, 64h + 64) of its region
+    // and writes the bf16 P^T / dS^T of its 64 queries (32 columns) back into the first half of
+    // those same columns, so no warpgroup overwrites columns the other still reads and the P
+    // phase needs no barrier; the MMAs that read P^T / dS^T as their A operand address each
+    // 16-query K step where it lies.  Otherwise the bf16 halves are packed into columns
+    // [32h, 32h + 32) behind a barrier.  The head-major kernels use own columns (+2 to +4 %);
+    // the packed-sequence kernel keeps the packed form, where the other addressing cost
+    // registers and measured 12 % slower.
+    __device__ static constexpr uint32_t bf16_col(bool own, int h) { return own ? 64u * h : 32u * h; }
+    __device__ static constexpr uint32_t a_col(bool own, int kk) {
+        return own ? (uint32_t)((kk / 4) * 64 + (kk % 4) * 8) : (uint32_t)(kk * 8);
     }
 };
 
@@ -121,6 +121,7 @@ __global__ void __launch_bounds__(512, 1)
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                   const BwdParams p) {
     using C = BwdCfg<D>;
+    constexpr bool OWN = !PACKED;  // own-column P^T / dS^T layout
     extern __shared__ __align__(1024) uint8_t smem[];
 
     const int warp = threadIdx.x / 32;
@@ -263,25 +264,25 @@ __global__ void __launch_bounds__(512, 1)
             return q < ext.Lq && in_bounds(p.err, (size_t)q_head(s) * p.N + q, 1, p.dbg.vec)
                        ? p.dOnorm[(size_t)q_head(s) * p.N + q] : -1.f;
         };
+        // (The packed-sequence kernel loads it in its own step: the prefetch cost it registers.)
+        constexpr bool prefetch = !PACKED;
         Step st{0, 0};
-        float norm = load_norm(st);
+        float norm = prefetch ? load_norm(st) : 0.f;
         for (int it = 0; it < n_it; ++it, st = next_step(st)) {
             const int q0 = q_block(st) * C::BM;
             // fixed-point scale of query q0 + r, shared by the drain warps; barrier 2 before the
             // reads and again after the last read of the step.  (A non-finite norm or bound
             // gives -1, which adds nothing; the dQ conversion reports it.)
+            if constexpr (!prefetch) norm = load_norm(st);
             s_scale[r] = norm >= 0.f ? fmaxf(fixed_point_scale(norm, factor), 0.f) : 0.f;
-            if (it + 1 < n_it) norm = load_norm(next_step(st));
+            if (prefetch && it + 1 < n_it) norm = load_norm(next_step(st));
             named_barrier(2, 128);
             const float* sc = s_scale;
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_dqfull, it & 1, p.timeout_ns, abort_flag));
-            constexpr int NV = (D == 128) ? 128 : 64;
-            uint32_t v[NV];
-            int* acc = p.dq_acc + ((size_t)q_head(st) * p.N_pad + q0) * D;
-            const bool acc_ok = in_bounds(p.err, ((size_t)q_head(st) * p.N_pad + q0) * D,
-                                          (size_t)C::BM * D, p.dbg.acc);
             if (ok) {
                 tc_fence_after();
+                constexpr int NV = (D == 128) ? 128 : 64;
+                uint32_t v[NV];
 #pragma unroll
                 for (int q = 0; q < NV / 32; ++q) tmem_ld32(tmem + lane_base + C::TM_B + 32 * q, v + 32 * q);
                 tmem_ld_wait();
@@ -289,7 +290,9 @@ __global__ void __launch_bounds__(512, 1)
                 for (int q = 0; q < NV / 32; ++q) reg_fence32(v + 32 * q);
                 tc_fence_before();
                 mbar_arrive(bar_dqempty);           // B may take the next dP^T
-                if (acc_ok) {
+                int* acc = p.dq_acc + ((size_t)q_head(st) * p.N_pad + q0) * D;
+                if (in_bounds(p.err, ((size_t)q_head(st) * p.N_pad + q0) * D, (size_t)C::BM * D,
+                              p.dbg.acc)) {
                     if constexpr (D == 128) {
                         // dQ^T: lane = feature r, column = query e; a warp instruction covers 32
                         // consecutive features of one query row: one 128-byte line.
@@ -419,7 +422,7 @@ __global__ void __launch_bounds__(512, 1)
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < C::BM / 16; ++kk)
-                mma_ts(tmem + C::TM_DV, tmem + C::TM_A + C::a_col(kk), dDO_mn + mnmaj(kk), idKV,
+                mma_ts(tmem + C::TM_DV, tmem + C::TM_A + C::a_col(OWN, kk), dDO_mn + mnmaj(kk), idKV,
                        (it > 0 || kk > 0) ? 1u : 0u);
             if (it + 1 < n_it) {
                 const int s1 = (it + 1) % C::QST;
@@ -434,7 +437,7 @@ __global__ void __launch_bounds__(512, 1)
                 // dK += dS^T Q, same shapes as dV (A = dS^T in tensor memory).
 #pragma unroll
                 for (int kk = 0; kk < C::BM / 16; ++kk)
-                    mma_ts(tmem + C::TM_DK, tmem + C::TM_B + C::a_col(kk), dQ_mn + mnmaj(kk), idKV,
+                    mma_ts(tmem + C::TM_DK, tmem + C::TM_B + C::a_col(OWN, kk), dQ_mn + mnmaj(kk), idKV,
                            (it > 0 || kk > 0) ? 1u : 0u);
                 tc_commit(&bar_qempty[s]);
             }
@@ -558,12 +561,12 @@ __global__ void __launch_bounds__(512, 1)
                 }
             }
             // (shared columns only) every S^T column read before P^T overwrites columns
-            if constexpr (!C::OWN_COLUMNS) named_barrier(1, 256);
+            if constexpr (!OWN) named_barrier(1, 256);
             if (ok) {
                 uint32_t pw[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) pw[e] = pack_bf16x2(P[2 * e], P[2 * e + 1]);
-                tmem_st32(tmem + lane_base + C::TM_A + C::bf16_col(h), pw);
+                tmem_st32(tmem + lane_base + C::TM_A + C::bf16_col(OWN, h), pw);
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(bar_pfull);
@@ -602,7 +605,7 @@ __global__ void __launch_bounds__(512, 1)
             named_barrier(1, 256);  // next step's lse / D stored; shared columns: dP^T read
             if (ok) {
                 // d = 128: dK reads dS^T from tensor memory; d = 64 reads the shared tile below.
-                if constexpr (D == 128) tmem_st32(tmem + lane_base + C::TM_B + C::bf16_col(h), dw);
+                if constexpr (D == 128) tmem_st32(tmem + lane_base + C::TM_B + C::bf16_col(OWN, h), dw);
                 // dS^T row r, queries [64h, 64h+64) = one 128-byte row of query chunk h; 16-byte
                 // unit u sits at position u ^ (r % 8) (the 128-byte swizzle the MMA reads).
 #pragma unroll
@@ -675,6 +678,7 @@ __global__ void __launch_bounds__(512, 1)
                           const __grid_constant__ CUtensorMap tmV,
                           const __grid_constant__ CUtensorMap tmDO, const BwdParams p) {
     using C = BwdCfg<D>;
+    constexpr bool OWN = true;  // own-column P^T / dS^T layout
     extern __shared__ __align__(1024) uint8_t smem[];
 
     const int warp = threadIdx.x / 32;
@@ -790,13 +794,10 @@ __global__ void __launch_bounds__(512, 1)
                 named_barrier(2, 128);
                 const float* sc = s_scale;
                 if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_dqfull, (gs + it) & 1, p.timeout_ns, abort_flag));
-                constexpr int NV = (D == 128) ? 128 : 64;
-                uint32_t v[NV];
-                int* acc = p.dq_acc + ((size_t)qh * p.N_pad + q0) * D;
-                const bool acc_ok =
-                    in_bounds(p.err, ((size_t)qh * p.N_pad + q0) * D, (size_t)C::BM * D, p.dbg.acc);
                 if (ok) {
                     tc_fence_after();
+                    constexpr int NV = (D == 128) ? 128 : 64;
+                    uint32_t v[NV];
 #pragma unroll
                     for (int q = 0; q < NV / 32; ++q) tmem_ld32(tmem + lane_base + C::TM_B + 32 * q, v + 32 * q);
                     tmem_ld_wait();
@@ -804,7 +805,8 @@ __global__ void __launch_bounds__(512, 1)
                     for (int q = 0; q < NV / 32; ++q) reg_fence32(v + 32 * q);
                     tc_fence_before();
                     mbar_arrive(bar_dqempty);  // B may take the next dP^T
-                    if (acc_ok) {
+                    int* acc = p.dq_acc + ((size_t)qh * p.N_pad + q0) * D;
+                    if (in_bounds(p.err, ((size_t)qh * p.N_pad + q0) * D, (size_t)C::BM * D, p.dbg.acc)) {
                         if constexpr (D == 128) {
 #pragma unroll
                             for (int e = 0; e < 128; e += 4) {
@@ -943,7 +945,7 @@ __global__ void __launch_bounds__(512, 1)
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < C::BM / 16; ++kk)
-                    mma_ts(tmem + C::TM_DV, tmem + C::TM_A + C::a_col(kk), dDO_mn + mnmaj(kk), idKV,
+                    mma_ts(tmem + C::TM_DV, tmem + C::TM_A + C::a_col(OWN, kk), dDO_mn + mnmaj(kk), idKV,
                            (it > 0 || kk > 0) ? 1u : 0u);
                 if (it + 1 < n_it) {
                     if (!(ok = mbar_wait(&bar_qfull[(g + 1) % C::QST], ((g + 1) / C::QST) & 1,
@@ -957,7 +959,7 @@ __global__ void __launch_bounds__(512, 1)
                 if constexpr (D == 128) {
 #pragma unroll
                     for (int kk = 0; kk < C::BM / 16; ++kk)
-                        mma_ts(tmem + C::TM_DK, tmem + C::TM_B + C::a_col(kk), dQ_mn + mnmaj(kk), idKV,
+                        mma_ts(tmem + C::TM_DK, tmem + C::TM_B + C::a_col(OWN, kk), dQ_mn + mnmaj(kk), idKV,
                                (it > 0 || kk > 0) ? 1u : 0u);
                     tc_commit(&bar_qempty[s]);
 #pragma unroll
@@ -1062,12 +1064,12 @@ __global__ void __launch_bounds__(512, 1)
                     }
                 }
                 // (shared columns only) every S^T column read before P^T overwrites columns
-                if constexpr (!C::OWN_COLUMNS) named_barrier(1, 256);
+                if constexpr (!OWN) named_barrier(1, 256);
                 if (ok) {
                     uint32_t pw[32];
 #pragma unroll
                     for (int e = 0; e < 32; ++e) pw[e] = pack_bf16x2(P[2 * e], P[2 * e + 1]);
-                    tmem_st32(tmem + lane_base + C::TM_A + C::bf16_col(h), pw);
+                    tmem_st32(tmem + lane_base + C::TM_A + C::bf16_col(OWN, h), pw);
                     tmem_st_wait();
                     tc_fence_before();
                     mbar_arrive(bar_pfull);
@@ -1102,7 +1104,7 @@ __global__ void __launch_bounds__(512, 1)
                 if (it + 1 < n_it) store_vectors(g + 1);
                 named_barrier(1, 256);  // next step's lse / D stored; shared columns: dP^T read
                 if (ok) {
-                    if constexpr (D == 128) tmem_st32(tmem + lane_base + C::TM_B + C::bf16_col(h), dw);
+                    if constexpr (D == 128) tmem_st32(tmem + lane_base + C::TM_B + C::bf16_col(OWN, h), dw);
 #pragma unroll
                     for (int v4 = 0; v4 < 8; ++v4)
                         *reinterpret_cast<uint4*>(ds_row + ((v4 ^ sw) << 4)) =
