@@ -128,13 +128,16 @@ KERNEL_SOURCES = {
 
 def main_kernels(w: workloads.Workload, num_sms: int) -> tuple[str, str]:
     """Names of the fused forward and backward kernels the library launches for `w`: the
-    persistent ones when every work unit costs the same (no causal mask, no key lengths) and
-    there are more units than SMs, the one-CTA-per-unit ones otherwise."""
+    persistent forward for launches without key lengths with more units than SMs and at most
+    32 key blocks per tile (causal or not), the persistent backward when every unit costs the
+    same (no causal mask either) and is at most 16 query steps long; the one-CTA-per-unit
+    kernels otherwise."""
     equal = not w.causal and w.pad_range is None
     fwd_units = -(-w.N // 256) * w.H * w.B
     bwd_units = -(-w.N // 128) * w.kv_heads * w.B
     steps = (w.H // w.kv_heads) * -(-w.N // 128)  # query steps of one backward unit
-    fwd = ("fa_fwd_persist_kernel" if equal and fwd_units > num_sms and -(-w.N // 128) <= 32
+    fwd = ("fa_fwd_persist_kernel"
+           if w.pad_range is None and fwd_units > num_sms and -(-w.N // 128) <= 32
            else "fa_fwd_kernel")
     bwd = ("fa_bwd_persist_kernel" if equal and bwd_units > num_sms and steps <= 16
            else "fa_bwd_kernel")

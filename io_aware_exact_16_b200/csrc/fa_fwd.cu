@@ -502,10 +502,12 @@ __global__ void __launch_bounds__(384, 1)
     }
 }
 
-// Persistent forward for launches whose work units all cost the same: head-major, no causal
-// mask, no per-sequence key lengths (every tile pair sees all N keys).  One CTA per SM walks
-// the units blockIdx.x, blockIdx.x + gridDim.x, ... (tile pair x of head bh, head by head, so
-// a few heads' K and V stay in L2).  Per key block the arithmetic is fa_fwd_kernel's; across
+// Persistent forward for head-major launches without per-sequence key lengths.  One CTA per SM
+// walks the units blockIdx.x, blockIdx.x + gridDim.x, ...: without a causal mask every unit
+// costs the same and they go head by head (tile pair x of head bh, so a few heads' K and V stay
+// in L2); with one, tile pair x needs x + 1 key blocks per tile and the units go heaviest
+// first across all heads (every head's last pair, then every head's second-to-last, ...), so
+// the static round robin ends on the lightest units.  Per key block the arithmetic is fa_fwd_kernel's; across
 // units the K/V ring and every barrier phase carry over, the Q tiles are reloaded as soon as the
 // previous unit's last score MMA has completed (bar_qempty), and a unit's epilogue overlaps the
 // next unit's Q load and first score MMAs.  A unit's first P V of tile t overwrites O_t only
@@ -523,8 +525,29 @@ __global__ void __launch_bounds__(384, 1)
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
     const int nx = (p.N + C::ROWS_PER_CTA - 1) / C::ROWS_PER_CTA;  // tile pairs per head
-    const int n_units = nx * p.B * p.H;
-    const int nblk = (p.N + C::BN - 1) / C::BN;  // key blocks of every query tile
+    const int BH = p.B * p.H;
+    const int n_units = nx * BH;
+    const int nblk = (p.N + C::BN - 1) / C::BN;  // key blocks of an unmasked query tile
+    // Unit lin: head bh and first query row; key blocks of tile t (rows up to q_base + 128 t
+    // + 127 see keys j < min(N, last row + 1) under the causal mask).
+    struct Unit {
+        int bh, q_base, n0, n1;
+    };
+    auto unit = [&](int lin) {
+        Unit u;
+        int x;
+        if (p.causal) {
+            x = nx - 1 - lin / BH;
+            u.bh = lin - (lin / BH) * BH;
+        } else {
+            u.bh = lin / nx;
+            x = lin - u.bh * nx;
+        }
+        u.q_base = x * C::ROWS_PER_CTA;
+        u.n0 = p.causal ? (min(p.N, u.q_base + C::BM) + C::BN - 1) / C::BN : nblk;
+        u.n1 = p.causal ? (min(p.N, u.q_base + 2 * C::BM) + C::BN - 1) / C::BN : nblk;
+        return u;
+    };
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_BAR);
     uint64_t* bar_q = bars;
@@ -587,8 +610,8 @@ __global__ void __launch_bounds__(384, 1)
             int uc = 0;  // units started
             bool ok = true;
             for (int lin = blockIdx.x; ok && lin < n_units; lin += gridDim.x, ++uc) {
-                const int bh = lin / nx;
-                const int q_base = (lin - bh * nx) * C::ROWS_PER_CTA;
+                const Unit u = unit(lin);
+                const int bh = u.bh, q_base = u.q_base;
                 const int bkv = (bh / p.H) * p.H_kv + (bh % p.H) / (p.H / p.H_kv);
                 if (uc > 0 && !(ok = mbar_wait(bar_qempty, (uc - 1) & 1, p.timeout_ns, abort_flag)))
                     break;
@@ -597,7 +620,7 @@ __global__ void __launch_bounds__(384, 1)
                     for (int c = 0; c < C::KCH; ++c)
                         tma_load_3d(smem + C::SMEM_Q + t * C::Q_TILE_BYTES + c * C::CHUNK_BYTES,
                                     &tmQ, bar_q, c * 64, q_base + t * C::BM, bh);
-                for (int j = 0; j < nblk; ++j, ++g) {
+                for (int j = 0; j < u.n1; ++j, ++g) {
                     const int s = g % C::STAGES;
                     const uint32_t ph = (g / C::STAGES) & 1;
                     if (!(ok = mbar_wait(&bar_kempty[s], ph ^ 1, p.timeout_ns, abort_flag))) break;
@@ -649,8 +672,8 @@ __global__ void __launch_bounds__(384, 1)
                            sdesc_sw128(va + kk * 2048, C::CHUNK_BYTES, 1024), idPV,
                            (accumulate || kk > 0) ? 1u : 0u);
             };
-            // cb = key blocks consumed before this one (the P barriers' phase), the same for
-            // both tiles here; accumulate unless this is a unit's first block.
+            // cb = key blocks tile t consumed before this one (the phase of its P barriers);
+            // accumulate unless this is a unit's first block.
             auto wait_issue_PV = [&](int t, int s, int cb, bool first) {
 #pragma unroll
                 for (int part = 0; part < C::P_PARTS; ++part) {
@@ -664,11 +687,15 @@ __global__ void __launch_bounds__(384, 1)
                 return true;
             };
             // Per unit: S_0(0) S_1(0), then per key block j: P V_0(j), S_0(j+1), P V_1(j),
-            // S_1(j+1); the commit after the unit's last score MMA releases the Q tiles.
+            // S_1(j+1), tile 0's products only for its n0 <= n1 blocks; the commit after the
+            // unit's last score MMA (S_1(n1 - 1)) releases the Q tiles.
             bool ok = true;
-            int g = 0;   // ring position of the unit's block 0 (= blocks consumed so far)
+            int g = 0;   // ring position of the unit's block 0 (= blocks loaded so far)
+            int c0 = 0;  // blocks tile 0 consumed in earlier units (its P barriers' phase)
             int uc = 0;  // units started
             for (int lin = blockIdx.x; ok && lin < n_units; lin += gridDim.x, ++uc) {
+                const Unit u = unit(lin);
+                const int n0 = u.n0, n1 = u.n1;
                 if (!(ok = mbar_wait(bar_q, uc & 1, p.timeout_ns, abort_flag))) break;
                 if (!(ok = mbar_wait(&bar_kfull[g % C::STAGES], (g / C::STAGES) & 1, p.timeout_ns,
                                      abort_flag)))
@@ -679,31 +706,36 @@ __global__ void __launch_bounds__(384, 1)
                 issue_S(1, g % C::STAGES);
                 tc_commit(&bar_sfull[1]);
                 tc_commit(&bar_kempty[g % C::STAGES]);
-                if (nblk == 1) tc_commit(bar_qempty);
-                for (int j = 0; ok && j < nblk; ++j) {
+                if (n1 == 1) tc_commit(bar_qempty);
+                for (int j = 0; ok && j < n1; ++j) {
                     const int gj = g + j, gn = gj + 1;
                     const int s = gj % C::STAGES, sn = gn % C::STAGES;
                     const uint32_t ph = (gj / C::STAGES) & 1, phn = (gn / C::STAGES) & 1;
                     if (!(ok = mbar_wait(&bar_vfull[s], ph, p.timeout_ns, abort_flag))) break;
-                    if (!(ok = wait_issue_PV(0, s, gj, j == 0))) break;
-                    tc_commit(&bar_ofull[0]);
-                    if (j + 1 < nblk) {
+                    if (j < n0) {
+                        if (!(ok = wait_issue_PV(0, s, c0 + j, j == 0))) break;
+                        tc_commit(&bar_ofull[0]);
+                    }
+                    if (j + 1 < n1) {
                         if (!(ok = mbar_wait(&bar_kfull[sn], phn, p.timeout_ns, abort_flag))) break;
                         tc_fence_after();
-                        issue_S(0, sn);
-                        tc_commit(&bar_sfull[0]);
+                        if (j + 1 < n0) {
+                            issue_S(0, sn);
+                            tc_commit(&bar_sfull[0]);
+                        }
                     }
                     if (!(ok = wait_issue_PV(1, s, gj, j == 0))) break;
                     tc_commit(&bar_ofull[1]);
                     tc_commit(&bar_vempty[s]);
-                    if (j + 1 < nblk) {
+                    if (j + 1 < n1) {
                         issue_S(1, sn);
                         tc_commit(&bar_sfull[1]);
                         tc_commit(&bar_kempty[sn]);
-                        if (j + 2 == nblk) tc_commit(bar_qempty);
+                        if (j + 2 == n1) tc_commit(bar_qempty);
                     }
                 }
-                g += nblk;
+                g += n1;
+                c0 += n0;
             }
             if (!ok) fail();
             tc_commit(bar_done);
@@ -719,13 +751,16 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t tS = tmem + lane_base + C::tm_s(t);
         const uint32_t tO = tmem + lane_base + C::tm_o(t);
         const float c = p.scale_log2;
-        const int lim = p.N;  // every key is visible
         bool ok = true;
         int cb = 0;  // key blocks processed (the phase of this tile's barriers)
         for (int lin = blockIdx.x; ok && lin < n_units; lin += gridDim.x) {
+            const Unit u = unit(lin);
+            const int nt = t ? u.n1 : u.n0;
+            // visible keys of this thread's row: j < lim (all N without the causal mask)
+            const int lim = p.causal ? min(p.N, u.q_base + t * C::BM + r + 1) : p.N;
             float m = -INFINITY;  // running max of S * c (log2 units), possibly stale by <= 8
             float l = 0.f;        // running sum of exp2(S * c - m)
-            for (int j = 0; j < nblk; ++j, ++cb) {
+            for (int j = 0; j < nt; ++j, ++cb) {
                 ok = mbar_wait(&bar_sfull[t], cb & 1, p.timeout_ns, abort_flag);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 tc_fence_after();
@@ -812,9 +847,9 @@ __global__ void __launch_bounds__(384, 1)
             if (ok) ok = mbar_wait(&bar_ofull[t], (cb - 1) & 1, p.timeout_ns, abort_flag);
             if (__all_sync(0xffffffffu, ok)) {
                 tc_fence_after();
-                const int lin_e = opaque(lin);  // recomputed here, not kept through the loop
-                const int bh = lin_e / nx;
-                const int row = (lin_e - bh * nx) * C::ROWS_PER_CTA + t * C::BM + r;
+                const Unit ue = unit(opaque(lin));  // recomputed here, not kept through the loop
+                const int bh = ue.bh;
+                const int row = ue.q_base + t * C::BM + r;
                 const float inv_l = l > 0.f ? 1.0f / l : 0.f;
                 const size_t o_off = ((size_t)bh * p.N + (row < p.N ? row : 0)) * D;
                 const bool in_range = row < p.N && in_bounds(p.err, o_off, D, p.dbg.q);
@@ -870,13 +905,13 @@ cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
         return e;
     const int nx = (p.N + C::ROWS_PER_CTA - 1) / C::ROWS_PER_CTA;
     const long long units = (long long)nx * p.H * B;
-    // Units of equal cost (head-major, no causal mask, no key lengths), more of them than SMs,
-    // and at most 32 key blocks long (N <= 4096; measured +3 to +30 % up to there, neutral
-    // to 2 % slower beyond): the persistent kernel, one CTA per SM.  Otherwise one CTA per
-    // unit in the heaviest-first order, which the hardware's CTA scheduler balances better
-    // than a static assignment when units differ in cost.
-    if (!PACKED && !p.causal && p.seqlens == nullptr && units > num_sms &&
-        (p.N + C::BN - 1) / C::BN <= 32) {
+    // Head-major launches without key lengths, more units than SMs and at most 32 key blocks
+    // per tile (N <= 4096): the persistent kernel, one CTA per SM.  Measured without the causal
+    // mask +3 to +30 % up to there and neutral to 2 % slower beyond; with it +34 / +25 / +10 / 0 %
+    // at N = 512 / 1024 / 2048 / 4096 (d = 128) and +35 / +23 / +11 / +5 % (d = 64).
+    // Otherwise one CTA per unit in the heaviest-first order.
+    const int nblk = (p.N + C::BN - 1) / C::BN;
+    if (!PACKED && p.seqlens == nullptr && units > num_sms && nblk <= 32) {
         fa_fwd_persist_kernel<D><<<num_sms, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
         return cudaGetLastError();
     }

@@ -94,14 +94,15 @@ def test_padded_keys_get_zero_gradient_and_garbage_changes_nothing():
         np.testing.assert_array_equal(a[name], b[name], err_msg=name)
 
 
+@pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("d", [64, 128])
-def test_persistent_and_per_unit_launches_are_bitwise_identical(d):
-    """Launches whose units all cost the same (head-major, non-causal, no key lengths, more
-    units than SMs) run the persistent forward and backward kernels; passing key lengths that
-    are all N selects the one-CTA-per-unit kernels for the same computation.  Both run the
-    same arithmetic in the same order, so every output must match bit for bit (and the oracle,
-    on two heads)."""
-    w = workloads.custom(4, 16, 1000, d, False, seed=3300 + d)
+def test_persistent_and_per_unit_launches_are_bitwise_identical(d, causal):
+    """Head-major launches without key lengths and with more units than SMs run the
+    persistent forward (causal or not) and, without the causal mask, the persistent backward;
+    passing key lengths that are all N selects the one-CTA-per-unit kernels for the same
+    computation.  Both run the same arithmetic in the same order, so every output must match
+    bit for bit (and the oracle, on two heads)."""
+    w = workloads.custom(4, 16, 1000, d, causal, seed=3300 + d + (7 if causal else 0))
     inp = workloads.make_inputs(w)
     _, a = run_fwd_bwd(w, inp)  # persistent (B*H*ceil(N/256) > SMs)
     full = torch.full((w.B,), w.N, dtype=torch.int32)
@@ -111,7 +112,7 @@ def test_persistent_and_per_unit_launches_are_bitwise_identical(d):
     for flat in workloads.seeded_sample(w.seed, w.B * w.H, 2):
         bi, h = divmod(flat, w.H)
         ref = oracle.head_bwd(inp.q[bi, h], inp.k[bi, h], inp.v[bi, h], inp.do[bi, h], w.scale,
-                              False)
+                              causal)
         assert_fwd_close(a["o"][bi, h], a["lse"][bi, h], ref["o"], ref["lse"], f"b{bi} h{h}")
         for name in ("dq", "dk", "dv"):
             assert_grad_close(a[name][bi, h], ref[name], name, f"b{bi} h{h}")
