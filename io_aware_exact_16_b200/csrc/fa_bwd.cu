@@ -92,11 +92,20 @@ struct BwdCfg {
     static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = SMEM_MISC + 16;  // tmem address, abort flag
     static constexpr int THREADS = 512;
-    // 2 x 136 (compute) + 88 (MMA / TMA) + 152 (drain) = 4 x 128 launched
-    static constexpr uint32_t REGS_COMPUTE = 136, REGS_OTHER = 88, REGS_DRAIN = 152;
+    // 2 x compute + MMA / TMA + drain = 4 x 128 launched.  The MMA thread spilled its operand
+    // descriptors at 88 registers, so every product it issued waited on local memory: 96 there
+    // measured +7 to +11 % (d = 128: 2 x 136 + 96 + 144; d = 64, whose drain holds half as
+    // many dQ values: 2 x 152 + 96 + 112).
+    static constexpr uint32_t REGS_COMPUTE = (D == 64) ? 152 : 136, REGS_OTHER = 96,
+                              REGS_DRAIN = (D == 64) ? 112 : 144;
     // The persistent kernel's MMA and TMA threads carry loop state across units and spill at
     // 88 registers: 2 x 128 + 104 + 152 there.
-    static constexpr uint32_t REGS_COMPUTE_PERSIST = 128, REGS_OTHER_PERSIST = 104;
+    static constexpr uint32_t REGS_COMPUTE_PERSIST = 128, REGS_OTHER_PERSIST = 104,
+                              REGS_DRAIN_PERSIST = 152;
+    static constexpr uint32_t REGS_LAUNCH = 65536 / THREADS;  // per thread at launch: 128
+    static_assert(2 * REGS_COMPUTE + REGS_OTHER + REGS_DRAIN == 4 * REGS_LAUNCH, "register split");
+    static_assert(2 * REGS_COMPUTE_PERSIST + REGS_OTHER_PERSIST + REGS_DRAIN_PERSIST == 4 * REGS_LAUNCH,
+                  "register split");
     static constexpr uint32_t TMEM_COLS = 512;
 
     static constexpr uint32_t TM_A = 0, TM_B = 128, TM_DV = 256, TM_DK = 256 + D;
@@ -249,7 +258,7 @@ __global__ void __launch_bounds__(512, 1)
     };
 
     if (warp >= 12) {
-        regs_increase<C::REGS_DRAIN>();
+        regs_set<C::REGS_DRAIN, C::REGS_LAUNCH>();
         // ------------------------------------------------------------ dQ drain
         const int r = threadIdx.x - 384;                // TMEM lane
         const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
@@ -335,7 +344,7 @@ __global__ void __launch_bounds__(512, 1)
         }
         if (!ok) fail();
     } else if (warp >= 8) {
-      regs_decrease<C::REGS_OTHER>();
+      regs_set<C::REGS_OTHER, C::REGS_LAUNCH>();
       if (warp == 9 && lane == 0) {
         // ------------------------------------------------------------ TMA producer
         prefetch_tensormap(&tmQ);
@@ -480,7 +489,7 @@ __global__ void __launch_bounds__(512, 1)
         mbar_wait_drain(bar_done, 0, p.timeout_ns);
       }
     } else {
-        regs_increase<C::REGS_COMPUTE>();
+        regs_set<C::REGS_COMPUTE, C::REGS_LAUNCH>();
         // ------------------------------------------------------------ compute warpgroups
         const int h = warp / 4;                          // query-column half
         const int r = threadIdx.x % 128;                 // TMEM lane
@@ -766,7 +775,7 @@ __global__ void __launch_bounds__(512, 1)
     };
 
     if (warp >= 12) {
-        regs_increase<C::REGS_DRAIN>();
+        regs_set<C::REGS_DRAIN_PERSIST, C::REGS_LAUNCH>();
         // ------------------------------------------------------------ dQ drain
         const int r = threadIdx.x - 384;  // TMEM lane
         const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
@@ -845,7 +854,7 @@ __global__ void __launch_bounds__(512, 1)
         }
         if (!ok) fail();
     } else if (warp >= 8) {
-      regs_decrease<C::REGS_OTHER_PERSIST>();
+      regs_set<C::REGS_OTHER_PERSIST, C::REGS_LAUNCH>();
       if (warp == 9 && lane == 0) {
         // ------------------------------------------------------------ TMA producer
         prefetch_tensormap(&tmQ);
@@ -992,7 +1001,7 @@ __global__ void __launch_bounds__(512, 1)
         mbar_wait_drain(bar_done, 0, p.timeout_ns);
       }
     } else {
-        regs_increase<C::REGS_COMPUTE_PERSIST>();
+        regs_set<C::REGS_COMPUTE_PERSIST, C::REGS_LAUNCH>();
         // ------------------------------------------------------------ compute warpgroups
         const int h = warp / 4;           // query-column half
         const int r = threadIdx.x % 128;  // TMEM lane

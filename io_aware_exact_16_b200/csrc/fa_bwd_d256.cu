@@ -62,7 +62,10 @@ struct Bwd256 {
     static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = SMEM_MISC + 16;  // tmem address, abort flag
     static constexpr int THREADS = 512;
-    static constexpr uint32_t REGS_COMPUTE = 136, REGS_OTHER = 88, REGS_DRAIN = 152;
+    // 2 x 136 + 104 (MMA / TMA; their threads spilled at 88) + 136 = 4 x 128 launched
+    static constexpr uint32_t REGS_COMPUTE = 136, REGS_OTHER = 104, REGS_DRAIN = 136;
+    static constexpr uint32_t REGS_LAUNCH = 65536 / THREADS;  // per thread at launch: 128
+    static_assert(2 * REGS_COMPUTE + REGS_OTHER + REGS_DRAIN == 4 * REGS_LAUNCH, "register split");
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t TM_A = 0, TM_B = 64, TM_DQ = 128, TM_DV = 256, TM_DK = 384;
     // Warpgroup h reads the fp32 S^T / dP^T columns [32h, 32h + 32) and writes the bf16 P^T /
@@ -188,7 +191,7 @@ __global__ void __launch_bounds__(512, 1)
     };
 
     if (warp >= 12) {
-        regs_increase<C::REGS_DRAIN>();
+        regs_set<C::REGS_DRAIN, C::REGS_LAUNCH>();
         // ------------------------------------------------------------ dQ drain
         const int r = threadIdx.x - 384;                // TMEM lane = feature r of the half
         const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
@@ -236,7 +239,7 @@ __global__ void __launch_bounds__(512, 1)
         }
         if (!ok) fail();
     } else if (warp >= 8) {
-      regs_decrease<C::REGS_OTHER>();
+      regs_set<C::REGS_OTHER, C::REGS_LAUNCH>();
       if (warp == 9 && lane == 0) {
         // ------------------------------------------------------------ TMA producer
         prefetch_tensormap(&tmQ);
@@ -334,7 +337,7 @@ __global__ void __launch_bounds__(512, 1)
         mbar_wait_drain(bar_done, 0, p.timeout_ns);
       }
     } else {
-        regs_increase<C::REGS_COMPUTE>();
+        regs_set<C::REGS_COMPUTE, C::REGS_LAUNCH>();
         // ------------------------------------------------------------ compute warpgroups
         const int h = warp / 4;                          // query-column half of a step
         const int r = threadIdx.x % 128;                 // TMEM lane = key row

@@ -25,7 +25,8 @@
 //   warp  9    TMA producer (one thread)
 //   warps 10-11 idle
 // The third warpgroup hands most of its registers to the two softmax warpgroups
-// (setmaxnreg: 56 + 2 x 224 per thread slot = 3 x 168 launched).
+// (setmaxnreg: 56 + 2 x 224 per thread slot = 3 x 168 launched; 72 + 2 x 216 in the packed-sequence
+// kernel, whose MMA thread spilled at 56).
 // Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+d) O1 [256+d,256+2d).
 // Shared memory: Q0, Q1, and a ring of K and V blocks, all 128-byte swizzled by TMA.
 #include "fa_internal.h"
@@ -66,6 +67,9 @@ struct FwdCfg {
     static constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;  // + alignment slack
     static constexpr int THREADS = 384;
     static constexpr uint32_t REGS_SOFTMAX = 224, REGS_OTHER = 56;
+    // packed sequences: 56 registers spilled the MMA thread's loop state (72 measured +6 %; the
+    // head-major kernels measured 2 % slower with it)
+    static constexpr uint32_t REGS_SOFTMAX_PACKED = 216, REGS_OTHER_PACKED = 72;
     // The persistent kernel's MMA and TMA threads carry loop state across units and spill at
     // 56 registers; there the split is 2 x 208 + 88 (the same 3 x 168 launched).
 #ifndef FA_FWD_PERSIST_REGS_SOFTMAX
@@ -73,6 +77,10 @@ struct FwdCfg {
 #endif
     static constexpr uint32_t REGS_SOFTMAX_PERSIST = FA_FWD_PERSIST_REGS_SOFTMAX;
     static constexpr uint32_t REGS_OTHER_PERSIST = 504 - 2 * REGS_SOFTMAX_PERSIST;
+    static constexpr uint32_t REGS_LAUNCH = 168;  // per thread at launch (65536 / 384, rounded to 8)
+    static_assert(2 * REGS_SOFTMAX + REGS_OTHER == 3 * REGS_LAUNCH, "register split");
+    static_assert(2 * REGS_SOFTMAX_PACKED + REGS_OTHER_PACKED == 3 * REGS_LAUNCH, "register split");
+    static_assert(2 * REGS_SOFTMAX_PERSIST + REGS_OTHER_PERSIST == 3 * REGS_LAUNCH, "register split");
     static constexpr uint32_t TMEM_COLS = 512;
     // tensor-memory column of S_t / O_t for query tile t
     __device__ static constexpr uint32_t tm_s(int t) { return t ? 128u : 0u; }
@@ -216,7 +224,7 @@ __global__ void __launch_bounds__(384, 1)
     };
 
     if (warp >= 8) {
-      regs_decrease<C::REGS_OTHER>();
+      regs_set<PACKED ? C::REGS_OTHER_PACKED : C::REGS_OTHER, C::REGS_LAUNCH>();
       if (warp == 9) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
@@ -347,7 +355,7 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
     } else {
-        regs_increase<C::REGS_SOFTMAX>();
+        regs_set<PACKED ? C::REGS_SOFTMAX_PACKED : C::REGS_SOFTMAX, C::REGS_LAUNCH>();
         // ------------------------------------------------------------ softmax warpgroups
         const int t = warp / 4;
         const int r = threadIdx.x % C::BM;
@@ -602,7 +610,7 @@ __global__ void __launch_bounds__(384, 1)
     };
 
     if (warp >= 8) {
-      regs_decrease<C::REGS_OTHER_PERSIST>();
+      regs_set<C::REGS_OTHER_PERSIST, C::REGS_LAUNCH>();
       if (warp == 9) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
@@ -747,7 +755,7 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
     } else {
-        regs_increase<C::REGS_SOFTMAX_PERSIST>();
+        regs_set<C::REGS_SOFTMAX_PERSIST, C::REGS_LAUNCH>();
         // ------------------------------------------------------------ softmax warpgroups
         const int t = warp / 4;
         const int r = threadIdx.x % C::BM;

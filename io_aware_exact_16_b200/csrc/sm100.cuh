@@ -281,6 +281,16 @@ template <uint32_t N>
 __device__ __forceinline__ void regs_decrease() {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
+// Moves this warpgroup's per-thread register count from LAUNCHED (the launch's allocation) to
+// TARGET: setmaxnreg.inc may not lower the count and .dec may not raise it, so the direction is
+// chosen here at compile time.  (An unchanged count still issues the .inc: it also tells the
+// register allocator the budget of the code that follows.)
+template <uint32_t TARGET, uint32_t LAUNCHED>
+__device__ __forceinline__ void regs_set() {
+    static_assert(TARGET % 8 == 0 && TARGET >= 24 && TARGET <= 256, "setmaxnreg count");
+    if constexpr (TARGET >= LAUNCHED) regs_increase<TARGET>();
+    else regs_decrease<TARGET>();
+}
 
 // ------------------------------------------------------------------ global memory helpers
 __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
